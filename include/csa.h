@@ -1,0 +1,245 @@
+/*
+ * csa.h -- C-ABI of the CSA2 FP4 compressed sparse-KV decode path (sm_100a).
+ *
+ * The method is the Compressed Sparse Attention 2 (CSA2) KV path of DeepSeek-V4.1-Flash, as three
+ * web pages describe it:
+ *   [rebasdaily] rebasdaily.com article on DeepSeek-V4.1-Flash KV compression, section
+ *                "同一份笔记，多层一起用" (layer modes Full / Reindex / Reuse; hierarchical sparse
+ *                indexer with a 2,048 x 8 = 16,384-position candidate pool; main KV in FP4, SWA KV
+ *                in FP8) and section "先让长输入少走一半路" (sliding-window attention branch).
+ *   [ailily]     ailily.cc article "每个 token 只占 890 字节", section 二 (mode table; one E4M3 scale
+ *                per 16 channels) and section 三 (range argument: sqrt(512) and 448 x 6 = 2688).
+ *   [yomxxx]     yomxxx.com long-form post on KV-cache compression limits, section 五 (attention
+ *                kernels need a fixed layout with addresses computed from the token index and
+ *                in-kernel parallel dequantisation).
+ *
+ * Conventions for every entry point
+ *   - All array arguments are DEVICE pointers unless marked "host".  The caller allocates and owns
+ *     every buffer; the library never allocates, frees or synchronises (except
+ *     csa_check_device_error, which synchronises the given stream).
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the legacy default stream)
+ *     and runs on the calling thread's current CUDA device.
+ *   - bf16 tensors are passed as uint16_t bit patterns.
+ *   - Every device pointer must be 16-byte aligned.
+ *   - Errors the host can see (null or misaligned pointers, unsupported sizes, too small a
+ *     workspace) return before anything is launched.  Launch failures return CSA_ERR_CUDA.
+ *     Errors in device-resident data (a page id, block id, slot or SWA row out of range, a
+ *     sequence longer than max_seq_len, an unsorted pool) are recorded in the workspace's status
+ *     word, the offending item is skipped, and csa_check_device_error reports them.
+ *   - Non-finite inputs give undefined (but memory-safe) results.
+ *
+ * KV layout (one per KV-producing Full layer), pages of 64 tokens:
+ *   codes     uint8 [num_pages][64][256]  E2M1 codes, channel 2i in the low nibble of byte i
+ *   scales    uint8 [num_pages][64][32]   E4M3 scale of channels 16g..16g+15
+ *   keys      uint8 [num_pages][64][128]  E4M3 indexer key
+ *   swa       uint8 [num_rows][128][512]  E4M3 sliding-window entry, position p at slot p % 128
+ *   swa_scale float [num_rows][128]       per-entry scale of the window entry
+ * A block is 8 consecutive positions; block b of a sequence lives in its page
+ * block_table[b / 8] at offsets 8*(b % 8) .. 8*(b % 8) + 7.
+ */
+#ifndef CSA_H
+#define CSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    CSA_OK = 0,
+    CSA_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, size out of range */
+    CSA_ERR_UNSUPPORTED = 2,  /* valid but unsupported configuration (e.g. H not in {16,32,64,128}) */
+    CSA_ERR_WORKSPACE = 3,    /* ws_bytes smaller than csa_workspace_bytes() requires */
+    CSA_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed */
+    CSA_ERR_DEVICE_DATA = 5,  /* device-resident metadata out of range (see csa_check_device_error) */
+    CSA_ERR_TIMEOUT = 6       /* a bounded device-side wait gave up */
+} csa_status;
+
+typedef enum { CSA_FULL = 0, CSA_REINDEX = 1, CSA_REUSE = 2 } csa_layer_mode;
+
+#define CSA_PAGE_TOKENS 64
+#define CSA_BLOCK_POSITIONS 8
+#define CSA_LATENT 512
+#define CSA_INDEX_HEADS 8
+#define CSA_INDEX_DIM 128
+#define CSA_WINDOW 128
+#define CSA_MAX_SEQ_LEN (1 << 24)
+#define CSA_MAX_TOPK 8192
+
+/* One KV-producing layer's caches.  All pointers device, caller-owned. */
+typedef struct {
+    uint8_t *codes;
+    uint8_t *scales;
+    uint8_t *keys;
+    uint8_t *swa;
+    float *swa_scale;
+    int32_t num_pages;
+    int32_t num_rows;
+} csa_kv_layer;
+
+/* One decode batch.  seq_len[b] >= 1 counts the current token; positions are 0 .. seq_len-1. */
+typedef struct {
+    int32_t B;                   /* host: number of sequences, 1 <= B <= 16384 */
+    const int32_t *seq_len;      /* device int32 [B], 1 <= seq_len[b] <= max_seq_len */
+    const int32_t *block_table;  /* device int32 [B][max_pages]: page id of each 64-token page */
+    int32_t max_pages;           /* host: row stride of block_table, >= ceil(max_seq_len / 64) */
+    const int32_t *swa_row;      /* device int32 [B]: the sequence's row of the SWA ring */
+    int32_t max_seq_len;         /* host: upper bound of seq_len[], sizes grids and workspace */
+} csa_batch;
+
+/* Size in bytes of the workspace the decode calls need for a batch of B sequences with H query
+ * heads, contexts up to max_seq_len, and selected-set capacities up to `cap` blocks (the largest
+ * Full Top-K or Reindex pool capacity used with this workspace).  Returns 0 for invalid sizes. */
+size_t csa_workspace_bytes(int32_t B, int32_t H, int32_t max_seq_len, int32_t cap);
+
+/* Bytes needed by calls that only report device-data errors (csa_kv_pack_fp4). */
+#define CSA_WORKSPACE_HEADER_BYTES 256
+
+/* Zero the workspace's status word.  Call once after allocating a workspace. */
+csa_status csa_workspace_init(void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Step 1 -- pack n tokens into one layer's caches ([rebasdaily] 同一份笔记，多层一起用: main KV in
+ * FP4, SWA KV stays FP8; [ailily] 二: one E4M3 scale per 16 channels).
+ *   latent   bf16 [n][512]  post-RMSNorm/RoPE latent (the value that serves as key and value)
+ *   idx_key  bf16 [n][128]  indexer key
+ *   slot     int64 [n]      destination page*64 + offset; must address a page < num_pages
+ *   swa_slot int32 [n]      row*128 + (position % 128) of the token's SWA entry, or -1 for none
+ * Per 16-channel group: a = max|x|, s = E4M3(a/6) (binary32 division, round-to-nearest-even,
+ * saturating), code = E2M1(x / s) (binary32 division, RNE, saturating, sign kept); s = 0 gives
+ * codes 0.  Key: E4M3 of each bf16 channel.  SWA: scale = max|x| / 448 (binary32),
+ * value = E4M3(x / scale).  ws needs CSA_WORKSPACE_HEADER_BYTES; a bad slot is skipped and
+ * recorded.  The results are bit-for-bit defined.
+ */
+csa_status csa_kv_pack_fp4(const csa_kv_layer *layer, const uint16_t *latent,
+                           const uint16_t *idx_key, const int64_t *slot, const int32_t *swa_slot,
+                           int32_t n, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Steps 2-3, Full layer -- score every block of every sequence and select its Top-k
+ * ([rebasdaily] 同一份笔记，多层一起用: a Full layer re-selects Top-K over the whole range; the
+ * first Full layer's scan builds the 2,048 x 8 candidate pool).
+ *   iq   bf16 [B][8][128]  indexer query, 8 heads
+ *   iw   float [B][8]      head weights
+ *   k    host, 1 <= k <= CSA_MAX_TOPK
+ *   out_blocks int32 [B][k]  selected block ids, ascending; entries past out_count are untouched
+ *   out_count  int32 [B]     min(k, ceil(seq_len/8))
+ * Score of position p: sum over heads h of w_h * ReLU(q_h . k_p), in binary32 in this order:
+ * per head, eight 16-dim FMA chains part_j, then ((p0+p4)+(p2+p6)) + ((p1+p5)+(p3+p7)), ReLU, and
+ * an FMA chain over h = 0..7.  Block score = max over its positions < seq_len.  Order: larger
+ * score first, then lower block id.  The selected set is bit-for-bit defined.
+ */
+csa_status csa_indexer_full(const csa_kv_layer *layer, const csa_batch *batch, const uint16_t *iq,
+                            const float *iw, int32_t k, int32_t *out_blocks, int32_t *out_count,
+                            void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Steps 2-3, Reindex layer -- re-score only the pool's blocks with this layer's own query and
+ * select the Top-k_r inside the pool ([rebasdaily] 同一份笔记，多层一起用: Reindex reuses the
+ * earlier layer's KV but re-evaluates which positions matter; later layers search only inside the
+ * pool).  `layer` is the KV of the Full layer that built the pool.
+ *   pool       int32 [B][pool_cap]  ascending block ids (a Full layer's output)
+ *   pool_count int32 [B]            valid entries per row, <= pool_cap
+ *   out_blocks int32 [B][k_r], out_count int32 [B] = min(k_r, pool_count)
+ * Same score, order and tie rule as csa_indexer_full.
+ */
+csa_status csa_indexer_reindex(const csa_kv_layer *layer, const csa_batch *batch,
+                               const uint16_t *iq, const float *iw, const int32_t *pool,
+                               const int32_t *pool_count, int32_t pool_cap, int32_t k_r,
+                               int32_t *out_blocks, int32_t *out_count, void *ws, size_t ws_bytes,
+                               void *stream);
+
+/*
+ * Step 2 alone -- block scores into a caller buffer (csa_indexer_full and csa_indexer_reindex run
+ * this and then csa_topk_blocks on workspace memory).  Full mode when pool is NULL: scores[b][v] for
+ * blocks v < ceil(seq_len/8); Reindex mode: scores[b][v] of pool[b][v] for v < pool_count[b].
+ *   scores float [B][score_stride], score_stride >= ceil(max_seq_len/8) (Full) or pool_cap (Reindex)
+ * Same score as csa_indexer_full; bit-for-bit defined.  Entries past each row's count are untouched.
+ */
+csa_status csa_indexer_block_scores(const csa_kv_layer *layer, const csa_batch *batch,
+                                    const uint16_t *iq, const float *iw, const int32_t *pool,
+                                    const int32_t *pool_count, int32_t pool_cap, float *scores,
+                                    int32_t score_stride, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Step 3 alone -- exact Top-k of block scores from csa_indexer_block_scores (same pool arguments):
+ * larger score first, then lower block id; the min(k, n) chosen block ids are written ascending.
+ * Bit-for-bit defined.  ws needs CSA_WORKSPACE_HEADER_BYTES.
+ */
+csa_status csa_topk_blocks(const csa_batch *batch, const float *scores, int32_t score_stride,
+                           const int32_t *pool, const int32_t *pool_count, int32_t pool_cap,
+                           int32_t k, int32_t *out_blocks, int32_t *out_count, void *ws,
+                           size_t ws_bytes, void *stream);
+
+/*
+ * Step 3, Reuse layer -- take the previous layer's selected set unchanged ([rebasdaily]
+ * 同一份笔记，多层一起用: Reuse keeps both the global KV and the earlier layer's Top-K positions).
+ * Copies prev_count[b] entries of each row and the counts; bytewise identical.
+ *   prev_blocks int32 [B][prev_cap], prev_count int32 [B] (each <= out_cap)
+ *   out_blocks  int32 [B][out_cap],  out_count  int32 [B]
+ */
+csa_status csa_index_reuse(int32_t B, const int32_t *prev_blocks, const int32_t *prev_count,
+                           int32_t prev_cap, int32_t *out_blocks, int32_t *out_count,
+                           int32_t out_cap, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Step 4 -- sparse decode attention over the selected FP4 entries and the FP8 window, merged
+ * through one softmax ([rebasdaily] 同一份笔记，多层一起用 and 先让长输入少走一半路; [yomxxx] 五:
+ * fixed layout, in-kernel parallel dequantisation).
+ *   q        bf16 [B][H][512], H in {16, 32, 64, 128}
+ *   sm_scale host, softmax temperature tau (1/sqrt(512) is the usual choice)
+ *   blocks   int32 [B][cap] selected block ids (< ceil(seq_len/8)), count int32 [B] <= cap
+ *   out      float [B][H][512], lse float [B][H]
+ * Segment E: the positions < seq_len of the selected blocks, value e2m1(code) * e4m3(scale)
+ * (exact).  Segment F: positions max(0, seq_len-128) .. seq_len-1 from the SWA ring row, value
+ * e4m3 * swa_scale.  A position in both segments counts once in each.  z = tau * q_h . value;
+ * out_h = softmax-weighted sum of values; lse_h = log-sum-exp of z.  Computed with fp16 operands
+ * (exact for these values) and fp32 accumulation; agrees with exact arithmetic to within
+ * 2e-3 of max|out| per sequence.
+ */
+csa_status csa_sparse_decode_attn(const csa_kv_layer *layer, const csa_batch *batch,
+                                  const uint16_t *q, int32_t H, float sm_scale,
+                                  const int32_t *blocks, const int32_t *count, int32_t cap,
+                                  float *out, float *lse, void *ws, size_t ws_bytes, void *stream);
+
+/* One decode step of one layer. */
+typedef struct {
+    csa_layer_mode mode;
+    const uint16_t *iq;          /* Full / Reindex: bf16 [B][8][128] */
+    const float *iw;             /* Full / Reindex: float [B][8] */
+    int32_t k;                   /* Full: Top-K; Reindex: k_r; ignored for Reuse */
+    const int32_t *prev_blocks;  /* Reindex: the pool; Reuse: the previous set */
+    const int32_t *prev_count;
+    int32_t prev_cap;
+    int32_t *blocks;             /* this layer's set, int32 [B][cap] (written) */
+    int32_t *count;              /* int32 [B] (written) */
+    int32_t cap;                 /* row stride of blocks; Full and Reindex require cap == k */
+    const uint16_t *q;           /* bf16 [B][H][512] */
+    int32_t H;
+    float sm_scale;
+    float *out;                  /* float [B][H][512] */
+    float *lse;                  /* float [B][H] */
+} csa_layer_step;
+
+/*
+ * Steps 2-4 for one layer in the given mode ([rebasdaily] 同一份笔记，多层一起用; [ailily] 二 mode
+ * table): Full = csa_indexer_full(k); Reindex = csa_indexer_reindex(prev, k); Reuse =
+ * csa_index_reuse(prev); then csa_sparse_decode_attn over this layer's set.  Reindex and Reuse
+ * layers pass the KV of the most recent Full layer.
+ */
+csa_status csa_decode_layer(const csa_kv_layer *layer, const csa_batch *batch,
+                            const csa_layer_step *step, void *ws, size_t ws_bytes, void *stream);
+
+/* Synchronise `stream`, read and clear the workspace status word.  Returns CSA_OK,
+ * CSA_ERR_DEVICE_DATA or CSA_ERR_TIMEOUT; *detail (host, may be NULL) receives the first
+ * offending index recorded. */
+csa_status csa_check_device_error(void *ws, void *stream, int64_t *detail);
+
+const char *csa_status_string(csa_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CSA_H */

@@ -1,0 +1,89 @@
+"""The C-ABI library without a GPU: it loads, exports every function include/csa.h declares, sizes
+workspaces, and rejects bad host arguments before touching the device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "csa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from fp4_compressed_sparse_kv_b200 import build, csa
+    build.build()
+    return csa.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(csa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ["csa_kv_pack_fp4", "csa_indexer_full", "csa_indexer_reindex", "csa_index_reuse",
+              "csa_sparse_decode_attn", "csa_decode_layer", "csa_workspace_bytes",
+              "csa_workspace_init", "csa_check_device_error", "csa_status_string"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from fp4_compressed_sparse_kv_b200 import csa
+    out = subprocess.run(["nm", "-D", "--defined-only", csa.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\sT\s(csa_\w+)", out))
+    for n in declared_functions():
+        assert n in exported, n
+        assert getattr(lib, n) is not None
+    assert set(csa.EXPORTS) <= exported
+
+
+def test_status_strings(lib):
+    for s in range(7):
+        assert lib.csa_status_string(s)
+    assert lib.csa_status_string(3) == b"workspace too small"
+
+
+def test_workspace_sizes(lib):
+    f = lib.csa_workspace_bytes
+    assert f(8, 64, 131072, 2048) > 0
+    assert f(8, 64, 131072, 2048) >= f(8, 64, 131072, 512) >= f(8, 16, 131072, 512)
+    assert f(1, 16, 4096, 64) > 256
+    # invalid sizes give 0
+    assert f(0, 64, 1000, 64) == 0
+    assert f(1, 24, 1000, 64) == 0
+    assert f(1, 64, 0, 64) == 0
+    assert f(1, 64, 1 << 25, 64) == 0
+    assert f(1, 64, 1000, 0) == 0
+    assert f(1, 64, 1000, 8193) == 0
+
+
+def test_bad_host_arguments_return_before_launch(lib):
+    from fp4_compressed_sparse_kv_b200 import csa
+    null = None
+    # null layer / batch
+    assert lib.csa_indexer_full(null, null, null, null, 64, null, null, null, 0, null) == 1
+    assert lib.csa_sparse_decode_attn(null, null, null, 64, ctypes.c_float(0.1), null, null, 64, null,
+                                      null, null, 0, null) == 1
+    assert lib.csa_index_reuse(0, null, null, 1, null, null, 1, null, 0, null) == 1
+    assert lib.csa_workspace_init(null, 256, null) == 1
+    assert lib.csa_check_device_error(null, null, null) == 1
+    # misaligned pointers are rejected too
+    fake = ctypes.c_void_p(0x1000)
+    odd = ctypes.c_void_p(0x1001)
+    layer = csa.KVLayerC(0x1000, 0x1000, odd.value, 0x1000, 0x1000, 4, 1)
+    assert lib.csa_kv_pack_fp4(ctypes.byref(layer), fake, fake, fake, null, 1, fake, 256, null) == 1
+    # n == 0 is a no-op
+    assert lib.csa_kv_pack_fp4(null, null, null, null, null, 0, null, 0, null) == 0
+
+
+def test_binding_refuses_host_tensors():
+    import torch
+    from fp4_compressed_sparse_kv_b200 import csa
+    with pytest.raises(ValueError):
+        csa._ptr(torch.zeros(4), "x")
