@@ -125,7 +125,7 @@ def source_sha(names):
 
 
 KERNEL_SOURCES = {"indexer_block_scores": ["indexer.cu", "common.cuh", "convert.cuh", "pipeline.cuh"],
-                  "sparse_decode_attn": ["attention_cc.cu", "attention_tc.cu", "attention_common.cuh",
+                  "sparse_decode_attn": ["attention_cc.cu", "attention_tc.cu", "attention_common.cuh", "tcgen05.cuh",
                                          "common.cuh", "convert.cuh"],
                   "topk_blocks": ["indexer.cu", "common.cuh"],
                   "kv_pack_fp4": ["pack.cu", "common.cuh", "convert.cuh"]}

@@ -194,34 +194,67 @@ cudaError_t launch_attn_cc(const AttnArgs &a, cudaStream_t st)
 
 // ------------------------------------------------------------------------------------------------
 // Split combine: out = sum_s e^{m_s - M} o_s / sum_s e^{m_s - M} l_s, lse = M + ln(sum ...).
+// One CTA per (head, sequence): the split weights are computed once into shared memory, then each
+// thread accumulates 4 channels with its loads of consecutive splits independent of one another.
 // ------------------------------------------------------------------------------------------------
+constexpr int kCombineMaxSplits = 1024;
+
 __global__ void __launch_bounds__(128) attn_combine_kernel(const float *__restrict__ part_o,
                                                           const float2 *__restrict__ part_ml, int splits, int H,
                                                           float *__restrict__ out, float *__restrict__ lse)
 {
-    const int h = blockIdx.x, b = blockIdx.y, t = threadIdx.x;
+    __shared__ float wgt[kCombineMaxSplits];
+    __shared__ float red[8];
+    const int h = blockIdx.x, b = blockIdx.y, t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const float2 *ml = part_ml + (size_t)b * splits * H + h;
     float M = -INFINITY;
-    for (int s = 0; s < splits; ++s) M = fmaxf(M, ml[(size_t)s * H].x);
+    for (int s = t; s < splits; s += 128) M = fmaxf(M, ml[(size_t)s * H].x);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    if (lane == 0) red[warp] = M;
+    __syncthreads();
+    M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
     float den = 0.f;
-    float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (M != -INFINITY) {
-        for (int s = 0; s < splits; ++s) {
-            const float2 v = ml[(size_t)s * H];
-            if (v.x == -INFINITY) continue;
-            const float wgt = expf(v.x - M);
-            den = fmaf(wgt, v.y, den);
-            const float4 o =
-                reinterpret_cast<const float4 *>(part_o + (((size_t)b * splits + s) * H + h) * kLatent)[t];
-            num.x = fmaf(wgt, o.x, num.x);
-            num.y = fmaf(wgt, o.y, num.y);
-            num.z = fmaf(wgt, o.z, num.z);
-            num.w = fmaf(wgt, o.w, num.w);
+    for (int s = t; s < splits; s += 128) {
+        const float2 v = ml[(size_t)s * H];
+        const float wv = (v.x == -INFINITY || M == -INFINITY) ? 0.f : expf(v.x - M);
+        wgt[s] = wv;
+        den = fmaf(wv, v.y, den);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    __syncthreads();
+    if (lane == 0) red[4 + warp] = den;
+    __syncthreads();
+    den = red[4] + red[5] + red[6] + red[7];
+    const float4 *po = reinterpret_cast<const float4 *>(part_o + ((size_t)b * splits * H + h) * kLatent) + t;
+    const size_t stride = (size_t)H * kLatent / 4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    int s = 0;
+    for (; s + 4 <= splits; s += 4) {
+        float4 o[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) o[q] = po[(size_t)(s + q) * stride];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float wv = wgt[s + q];
+            acc.x = fmaf(wv, o[q].x, acc.x);
+            acc.y = fmaf(wv, o[q].y, acc.y);
+            acc.z = fmaf(wv, o[q].z, acc.z);
+            acc.w = fmaf(wv, o[q].w, acc.w);
         }
+    }
+    for (; s < splits; ++s) {
+        const float4 o = po[(size_t)s * stride];
+        const float wv = wgt[s];
+        acc.x = fmaf(wv, o.x, acc.x);
+        acc.y = fmaf(wv, o.y, acc.y);
+        acc.z = fmaf(wv, o.z, acc.z);
+        acc.w = fmaf(wv, o.w, acc.w);
     }
     const float inv = den > 0.f ? 1.f / den : 0.f;
     reinterpret_cast<float4 *>(out + ((size_t)b * H + h) * kLatent)[t] =
-        make_float4(num.x * inv, num.y * inv, num.z * inv, num.w * inv);
+        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
     if (t == 0) lse[(size_t)b * H + h] = den > 0.f ? M + logf(den) : -INFINITY;
 }
 

@@ -23,7 +23,7 @@ constexpr int kWindow = CSA_WINDOW;
 // Workspace: [0, 256) status header; then block scores; then attention split partials.
 // ------------------------------------------------------------------------------------------------
 constexpr size_t kHeaderBytes = CSA_WORKSPACE_HEADER_BYTES;
-constexpr int kTargetCtas = 2 * 148;        // attention work items per step (2 per SM)
+constexpr int kNumSms = 148;                // B200 SM count, used to size the attention split
 constexpr int kAttnUnit = 8;                // entries per attention work unit (one block)
 constexpr int kWindowUnits = kWindow / kAttnUnit;
 
@@ -39,13 +39,16 @@ struct WsLayout {
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Attention split count per sequence: enough work items to fill the GPU, never more than the
-// sequence's largest number of 8-entry units (selected blocks plus the window).
+// Attention split count per sequence: about one wave of CTAs over the GPU (one CTA per SM for the
+// tensor-core kernel, whose 128-entry tiles fill the SM; two for the CUDA-core kernel), never more
+// than the sequence's largest number of tiles (selected blocks plus the window).
 inline int attn_splits(int B, int cap, int units_per_tile)
 {
     int max_units = cap + kWindowUnits;
     int max_tiles = (max_units + units_per_tile - 1) / units_per_tile;
-    int s = (kTargetCtas + B - 1) / B;
+    const int target = units_per_tile >= 16 ? kNumSms : 2 * kNumSms;
+    int s = target / B;
+    if (s < 1) s = 1;
     if (s > max_tiles) s = max_tiles;
     if (s < 1) s = 1;
     return s;

@@ -14,22 +14,24 @@
 namespace csa {
 
 // ------------------------------------------------------------------------------------------------
-// Block scoring.  Persistent CTAs; a work item is 8 consecutive "virtual" blocks of one sequence:
-// in Full mode virtual block v is block v (8 blocks = one 64-token page); in Reindex mode it is
-// pool[b][v].  A producer warp gathers each item's 8 x 1 KB key blocks into a shared-memory ring
-// with 1-D bulk copies; 8 consumer warps each score one block.  Consumer lane (g, j) = (lane/8,
-// lane%8) holds dims 16j..16j+15 of all 8 query heads in registers and takes key g of each group
-// of 4, so one 16-byte shared load feeds 128 FMAs.  The 8 per-lane partials per head are combined
-// by a 3-step xor reduce-scatter (distances 4, 2, 1) that forms exactly
-// ((p0+p4)+(p2+p6)) + ((p1+p5)+(p3+p7)) in every lane, up to the commutativity of each addition.
+// Block scoring.  Persistent CTAs of 8 warps; a work item is 8 consecutive "virtual" blocks of one
+// sequence (in Full mode virtual block v is block v, so an item is one 64-token page; in Reindex
+// mode it is pool[b][v]) and warp w always takes virtual block w of each item.  Every warp runs its
+// own pipeline: lane 0 resolves the block's page a few items ahead and bulk-copies its 1 KB of keys
+// into the warp's shared-memory ring; no warp ever waits for another.
+//
+// Lane (g, j) = (lane/8, lane%8) holds dims 16j..16j+15 of all 8 query heads in registers and takes
+// key g of each group of 4.  Lane j keeps head s^j in register slot s, so the 3-step xor
+// reduce-scatter (distances 4, 2, 1) needs no selects and leaves head j in lane j, having formed
+// exactly ((p0+p4)+(p2+p6)) + ((p1+p5)+(p3+p7)) up to the commutativity of each addition.  The
+// 16-term chains run as packed fma.rn.f32x2 over head pairs: two independent IEEE FMAs each.
 // ------------------------------------------------------------------------------------------------
-constexpr int kScoreStages = 8;
-constexpr int kScoreConsumers = 8;
-constexpr int kScoreThreads = (kScoreConsumers + 1) * 32;
-constexpr int kBlockBytes = kBlock * kIdxDim;              // 1 KB of keys per block
-constexpr int kStageBytes = kScoreConsumers * kBlockBytes;  // 8 KB per stage
-constexpr int kBlkEmpty = -2;                               // virtual block past the end
-constexpr int kBlkBad = -1;                                 // invalid metadata (reported)
+constexpr int kScoreWarps = 8;
+constexpr int kScoreThreads = kScoreWarps * 32;
+constexpr int kScoreStages = 6;
+constexpr int kBlockBytes = kBlock * kIdxDim;   // 1 KB of keys per block
+constexpr int kBlkEmpty = -2;                    // virtual block past the end
+constexpr int kBlkBad = -1;                      // invalid metadata (reported)
 
 struct ScoreArgs {
     const uint8_t *keys;
@@ -50,61 +52,74 @@ struct ScoreArgs {
     void *ws;
 };
 
-struct StageMeta {
+constexpr int kMetaRing = 64;   // per-warp ring of resolved items (>= 32 + kScoreStages)
+
+struct ItemMeta {
+    const uint8_t *src;   // the block's 1 KB of keys, or null
     int b;
     int L;
-    int blk[kScoreConsumers];
+    int blk;
+    int v;
 };
 
 struct ScoreSmem {
-    alignas(128) uint8_t stage[kScoreStages][kStageBytes];
-    StageMeta meta[kScoreStages];
-    uint64_t full[kScoreStages];
-    uint64_t empty[kScoreStages];
+    alignas(128) uint8_t stage[kScoreWarps][kScoreStages][kBlockBytes];
+    ItemMeta meta[kScoreWarps][kMetaRing];
+    uint64_t full[kScoreWarps][kScoreStages];
     int abort_flag;
 };
 
-__device__ __forceinline__ float score_key(const float (&q)[8][16], const float (&w)[8], uint4 kr, int lane)
+__device__ __forceinline__ unsigned long long f2_pack(float lo, float hi)
 {
-    const int j = lane & 7;
-    float k[16];
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ void f2_unpack(unsigned long long v, float &lo, float &hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+__device__ __forceinline__ unsigned long long ffma2(unsigned long long a, unsigned long long b, unsigned long long c)
+{
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+// Score of the key whose dims 16j..16j+15 this lane holds in kr.  q2[s2][t] = (q[h(2 s2)][16j+t],
+// q[h(2 s2+1)][16j+t]) with h(s) = s ^ j.
+__device__ __forceinline__ float score_key(const unsigned long long (&q2)[4][16], const float (&w)[8], uint4 kr,
+                                           int lane)
+{
+    unsigned long long k2[16];
     const uint32_t kw[4] = {kr.x, kr.y, kr.z, kr.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const uint32_t lo = e4m3x2_to_f16x2((uint16_t)(kw[i] & 0xFFFF));
         const uint32_t hi = e4m3x2_to_f16x2((uint16_t)(kw[i] >> 16));
-        k[4 * i + 0] = h_lo(lo);
-        k[4 * i + 1] = h_hi(lo);
-        k[4 * i + 2] = h_lo(hi);
-        k[4 * i + 3] = h_hi(hi);
+        const float k0 = h_lo(lo), k1 = h_hi(lo), k2v = h_lo(hi), k3 = h_hi(hi);
+        k2[4 * i + 0] = f2_pack(k0, k0);
+        k2[4 * i + 1] = f2_pack(k1, k1);
+        k2[4 * i + 2] = f2_pack(k2v, k2v);
+        k2[4 * i + 3] = f2_pack(k3, k3);
     }
-    float part[8];
+    float p[8];
 #pragma unroll
-    for (int h = 0; h < 8; ++h) {
-        float p = 0.f;
+    for (int s2 = 0; s2 < 4; ++s2) {
+        unsigned long long acc = 0ull;   // (+0, +0)
 #pragma unroll
-        for (int t = 0; t < 16; ++t) p = __fmaf_rn(q[h][t], k[t], p);
-        part[h] = p;
+        for (int t = 0; t < 16; ++t) acc = ffma2(q2[s2][t], k2[t], acc);
+        f2_unpack(acc, p[2 * s2], p[2 * s2 + 1]);
     }
-    // reduce-scatter over the 8 lanes of this key: lane j ends with head j
-    const bool up4 = j & 4, up2 = j & 2, up1 = j & 1;
     float a[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float send = up4 ? part[i] : part[4 + i];
-        const float keep = up4 ? part[4 + i] : part[i];
-        a[i] = __fadd_rn(keep, __shfl_xor_sync(0xffffffffu, send, 4));
-    }
+    for (int i = 0; i < 4; ++i) a[i] = __fadd_rn(p[i], __shfl_xor_sync(0xffffffffu, p[4 + i], 4));
     float c[2];
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const float send = up2 ? a[i] : a[2 + i];
-        const float keep = up2 ? a[2 + i] : a[i];
-        c[i] = __fadd_rn(keep, __shfl_xor_sync(0xffffffffu, send, 2));
-    }
-    const float send = up1 ? c[0] : c[1];
-    const float keep = up1 ? c[1] : c[0];
-    const float d = __fadd_rn(keep, __shfl_xor_sync(0xffffffffu, send, 1));
+    for (int i = 0; i < 2; ++i) c[i] = __fadd_rn(a[i], __shfl_xor_sync(0xffffffffu, a[2 + i], 2));
+    const float d = __fadd_rn(c[0], __shfl_xor_sync(0xffffffffu, c[1], 1));
     const float r = d > 0.f ? d : 0.f;
     float score = 0.f;
     const int base = lane & ~7;
@@ -121,179 +136,181 @@ __global__ void __launch_bounds__(kScoreThreads, 1) block_score_kernel(ScoreArgs
     const long long total = (long long)a.B * a.items_per_seq;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kScoreStages; ++s) {
-            mbar_init(&sm.full[s], 1);
-            mbar_init(&sm.empty[s], kScoreConsumers);
-        }
+        for (int w = 0; w < kScoreWarps; ++w)
+            for (int st = 0; st < kScoreStages; ++st) mbar_init(&sm.full[w][st], 1);
         sm.abort_flag = 0;
         fence_mbar_init();
     }
     __syncthreads();
 
-    if (warp == kScoreConsumers) {
-        // ---------------- producer ----------------
-        if (lane == 0) {
-            long long k = 0;
-            for (long long item = blockIdx.x; item < total; item += gridDim.x, ++k) {
-                const int st = (int)(k % kScoreStages);
-                const uint32_t ph = (uint32_t)((k / kScoreStages) & 1);
-                if (!mbar_wait(&sm.empty[st], ph ^ 1u, &sm.abort_flag, a.ws, item)) break;
-                const int b = (int)(item / a.items_per_seq);
-                const int grp = (int)(item % a.items_per_seq);
-                StageMeta &m = sm.meta[st];
-                const int L = a.seq_len[b];
-                m.b = b;
-                m.L = L;
-                int blks[kScoreConsumers];
-                uint32_t bytes = 0;
-                const bool L_ok = L >= 1 && L <= a.max_seq_len;
-                if (!L_ok && grp == 0) report(a.ws, CSA_ERR_DEVICE_DATA, b);
-                int nvb = 0;
-                if (L_ok) {
-                    nvb = a.pool ? a.pool_count[b] : (L + kBlock - 1) / kBlock;
-                    if (a.pool && (nvb < 0 || nvb > a.pool_cap)) {
-                        if (grp == 0) report(a.ws, CSA_ERR_DEVICE_DATA, b);
-                        nvb = 0;
-                    }
-                }
-                const int nb = (L + kBlock - 1) / kBlock;
-#pragma unroll
-                for (int w = 0; w < kScoreConsumers; ++w) {
-                    const int v = grp * kScoreConsumers + w;
-                    int blk = kBlkEmpty;
-                    if (v < nvb) {
-                        blk = a.pool ? a.pool[(size_t)b * a.pool_cap + v] : v;
-                        if (a.pool && v > 0 && a.pool[(size_t)b * a.pool_cap + v - 1] >= blk)
-                            report(a.ws, CSA_ERR_DEVICE_DATA, (long long)b * a.pool_cap + v);
-                        if (blk < 0 || blk >= nb) {
-                            report(a.ws, CSA_ERR_DEVICE_DATA, (long long)b * a.pool_cap + v);
-                            blk = kBlkBad;
-                        } else {
-                            const int page = a.block_table[(size_t)b * a.max_pages + blk / kBlocksPerPage];
-                            if (page < 0 || page >= a.num_pages) {
-                                report(a.ws, CSA_ERR_DEVICE_DATA, (long long)b * a.max_pages + blk / kBlocksPerPage);
-                                blk = kBlkBad;
-                            } else {
-                                bytes += kBlockBytes;
-                            }
-                        }
-                    }
-                    blks[w] = blk;
-                    m.blk[w] = blk;
-                }
-                if (bytes == 0) {
-                    mbar_arrive(&sm.full[st]);
-                } else {
-                    mbar_arrive_expect_tx(&sm.full[st], bytes);
-#pragma unroll
-                    for (int w = 0; w < kScoreConsumers; ++w) {
-                        const int blk = blks[w];
-                        if (blk < 0) continue;
-                        const int page = a.block_table[(size_t)b * a.max_pages + blk / kBlocksPerPage];
-                        const uint8_t *src =
-                            a.keys + ((size_t)page * kPage + (size_t)(blk % kBlocksPerPage) * kBlock) * kIdxDim;
-                        bulk_g2s(sm.stage[st] + w * kBlockBytes, src, kBlockBytes, &sm.full[st]);
-                    }
+    // ---- metadata of this warp's block of items k0 .. k0+31, one item per lane, loads in parallel
+    auto resolve32 = [&](long long k0) {
+        const long long k = k0 + lane;
+        const long long item = blockIdx.x + k * (long long)gridDim.x;
+        ItemMeta m{nullptr, 0, 0, kBlkEmpty, 0};
+        if (item < total) {
+            const int b = (int)(item / a.items_per_seq);
+            const int grp = (int)(item % a.items_per_seq);
+            const int L = a.seq_len[b];
+            int nvb = 0;
+            if (L < 1 || L > a.max_seq_len) {
+                if (grp == 0 && warp == 0) report(a.ws, CSA_ERR_DEVICE_DATA, b);
+            } else {
+                nvb = a.pool ? a.pool_count[b] : (L + kBlock - 1) / kBlock;
+                if (a.pool && (nvb < 0 || nvb > a.pool_cap)) {
+                    if (grp == 0 && warp == 0) report(a.ws, CSA_ERR_DEVICE_DATA, b);
+                    nvb = 0;
                 }
             }
-            // no copy may still be landing in shared memory when the CTA exits
-            const long long first = k > kScoreStages ? k - kScoreStages : 0;
-            for (long long kk = first; kk < k; ++kk) {
-                volatile int no_abort = 0;
-                mbar_wait(&sm.full[kk % kScoreStages], (uint32_t)((kk / kScoreStages) & 1), &no_abort, a.ws, -1);
+            const int v = grp * kScoreWarps + warp;
+            const int nb = (L + kBlock - 1) / kBlock;
+            m.b = b;
+            m.L = L;
+            m.v = v;
+            if (v < nvb) {
+                int blk = a.pool ? a.pool[(size_t)b * a.pool_cap + v] : v;
+                if (a.pool && v > 0 && a.pool[(size_t)b * a.pool_cap + v - 1] >= blk)
+                    report(a.ws, CSA_ERR_DEVICE_DATA, (long long)b * a.pool_cap + v);
+                if (blk < 0 || blk >= nb) {
+                    report(a.ws, CSA_ERR_DEVICE_DATA, (long long)b * a.pool_cap + v);
+                    blk = kBlkBad;
+                } else {
+                    const int page = a.block_table[(size_t)b * a.max_pages + blk / kBlocksPerPage];
+                    if (page < 0 || page >= a.num_pages) {
+                        report(a.ws, CSA_ERR_DEVICE_DATA, (long long)b * a.max_pages + blk / kBlocksPerPage);
+                        blk = kBlkBad;
+                    } else {
+                        m.src = a.keys + ((size_t)page * kPage + (size_t)(blk % kBlocksPerPage) * kBlock) * kIdxDim;
+                    }
+                }
+                m.blk = blk;
             }
         }
-    } else {
-        // ---------------- consumers ----------------
-        float q[8][16];
-        float w[8];
-        int cur_b = -1;
-        long long k = 0;
-        for (long long item = blockIdx.x; item < total; item += gridDim.x, ++k) {
-            const int st = (int)(k % kScoreStages);
-            const uint32_t ph = (uint32_t)((k / kScoreStages) & 1);
-            if (!mbar_wait(&sm.full[st], ph, &sm.abort_flag, a.ws, item)) break;
-            const StageMeta &m = sm.meta[st];
-            const int b = m.b, L = m.L;
-            const int blk = m.blk[warp];
-            if (blk >= 0) {
-                if (b != cur_b) {
-                    const int j = lane & 7;
-#pragma unroll
-                    for (int h = 0; h < 8; ++h) {
-                        const uint4 *src =
-                            reinterpret_cast<const uint4 *>(a.iq + ((size_t)b * kIdxHeads + h) * kIdxDim + 16 * j);
-                        const uint4 u0 = src[0], u1 = src[1];
-                        const uint32_t uw[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            q[h][2 * i] = bf16_lo(uw[i]);
-                            q[h][2 * i + 1] = bf16_hi(uw[i]);
-                        }
-                        w[h] = a.iw[(size_t)b * kIdxHeads + h];
-                    }
-                    cur_b = b;
-                }
-                const uint8_t *sp = sm.stage[st] + warp * kBlockBytes;
-                const int g = lane >> 3, j = lane & 7;
-                float best = -INFINITY;
-#pragma unroll
-                for (int it = 0; it < 2; ++it) {
-                    const int kk = it * 4 + g;
-                    const uint4 kr = *reinterpret_cast<const uint4 *>(sp + kk * kIdxDim + 16 * j);
-                    const float s = score_key(q, w, kr, lane);
-                    if (blk * kBlock + kk < L) best = fmaxf(best, s);
-                }
-                best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, 8));
-                best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, 16));
-                if (lane == 0) {
-                    const int v = (int)(item % a.items_per_seq) * kScoreConsumers + warp;
-                    a.scores[(size_t)b * a.score_stride + v] = best;
-                }
-            } else if (blk == kBlkBad && lane == 0) {
-                const int v = (int)(item % a.items_per_seq) * kScoreConsumers + warp;
-                a.scores[(size_t)b * a.score_stride + v] = -INFINITY;
-            }
+        sm.meta[warp][k % kMetaRing] = m;
+    };
+    // lane 0: start the copy of item k's block into stage k % kScoreStages
+    auto issue = [&](long long k) {
+        const long long item = blockIdx.x + k * (long long)gridDim.x;
+        if (item >= total) return;
+        const int st = (int)(k % kScoreStages);
+        const ItemMeta &m = sm.meta[warp][k % kMetaRing];
+        if (m.src) {
+            fence_async_smem();   // this warp's earlier reads of the stage precede the copy into it
+            mbar_arrive_expect_tx(&sm.full[warp][st], kBlockBytes);
+            bulk_g2s(sm.stage[warp][st], m.src, kBlockBytes, &sm.full[warp][st]);
+        } else {
+            mbar_arrive(&sm.full[warp][st]);
+        }
+    };
+
+    resolve32(0);
+    __syncwarp();
+    if (lane == 0)
+        for (long long k = 0; k < kScoreStages - 1; ++k) issue(k);
+    __syncwarp();
+
+    unsigned long long q2[4][16];
+    float w[8];
+    int cur_b = -1;
+    const int g = lane >> 3, j = lane & 7;
+    long long k = 0;
+    for (long long item = blockIdx.x; item < total; item += gridDim.x, ++k) {
+        const long long kn = k + kScoreStages - 1;   // the item whose copy starts now
+        if ((kn & 31) == 0) {
+            resolve32(kn);
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.empty[st]);
+        }
+        if (lane == 0) issue(kn);
+        const int st = (int)(k % kScoreStages);
+        if (!warp_wait(&sm.full[warp][st], (uint32_t)((k / kScoreStages) & 1), &sm.abort_flag, a.ws, item)) break;
+        const ItemMeta m = sm.meta[warp][k % kMetaRing];
+        if (m.blk >= 0) {
+            if (m.b != cur_b) {
+                cur_b = m.b;
+#pragma unroll
+                for (int s2 = 0; s2 < 4; ++s2) {
+                    const int h0 = (2 * s2) ^ j, h1 = (2 * s2 + 1) ^ j;
+                    const uint4 *r0 =
+                        reinterpret_cast<const uint4 *>(a.iq + ((size_t)m.b * kIdxHeads + h0) * kIdxDim + 16 * j);
+                    const uint4 *r1 =
+                        reinterpret_cast<const uint4 *>(a.iq + ((size_t)m.b * kIdxHeads + h1) * kIdxDim + 16 * j);
+                    const uint4 x0 = r0[0], x1 = r0[1], y0 = r1[0], y1 = r1[1];
+                    const uint32_t xw[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                    const uint32_t yw[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        q2[s2][2 * i] = f2_pack(bf16_lo(xw[i]), bf16_lo(yw[i]));
+                        q2[s2][2 * i + 1] = f2_pack(bf16_hi(xw[i]), bf16_hi(yw[i]));
+                    }
+                }
+#pragma unroll
+                for (int h = 0; h < 8; ++h) w[h] = a.iw[(size_t)m.b * kIdxHeads + h];
+            }
+            const uint8_t *sp = sm.stage[warp][st];
+            const uint4 kr0 = *reinterpret_cast<const uint4 *>(sp + g * kIdxDim + 16 * j);
+            const uint4 kr1 = *reinterpret_cast<const uint4 *>(sp + (4 + g) * kIdxDim + 16 * j);
+            const float s0 = score_key(q2, w, kr0, lane);
+            const float s1 = score_key(q2, w, kr1, lane);
+            float best = -INFINITY;
+            if (m.blk * kBlock + g < m.L) best = s0;
+            if (m.blk * kBlock + 4 + g < m.L) best = fmaxf(best, s1);
+            best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, 8));
+            best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, 16));
+            if (lane == 0) a.scores[(size_t)m.b * a.score_stride + m.v] = best;
+        } else if (m.blk == kBlkBad && lane == 0) {
+            a.scores[(size_t)m.b * a.score_stride + m.v] = -INFINITY;
+        }
+        __syncwarp();
+    }
+    // no copy may still be landing in shared memory when the CTA exits: wait for every stage this
+    // warp started (k counts the items consumed; issue() ran up to k + kScoreStages - 2)
+    if (lane == 0) {
+        for (long long kk = k; kk < k + kScoreStages - 1; ++kk) {
+            const long long item = blockIdx.x + kk * (long long)gridDim.x;
+            if (item >= total) break;
+            volatile int no_abort = 0;
+            mbar_wait(&sm.full[warp][kk % kScoreStages], (uint32_t)((kk / kScoreStages) & 1), &no_abort, a.ws, -1);
         }
     }
-    __syncthreads();
+    __syncwarp();
 }
 
 // ------------------------------------------------------------------------------------------------
-// Exact Top-K of one sequence's n candidate scores: radix select of the k-th largest order key in
-// four 8-bit passes (keys cached in shared memory when they fit), then one ascending pass that
-// keeps every key above the threshold and the lowest-indexed ties, written in index order.
+// Exact Top-K of one sequence's n candidate scores, one CTA per sequence.  Scores become order keys
+// (a total order on floats); keys are cached in shared memory when they fit.  The bits that every
+// key shares (the common prefix of the minimum and maximum key) are skipped; the rest are resolved
+// MSB first in digits of up to 8 bits with per-warp shared-memory histograms, giving the exact k-th
+// largest key T and the number need_eq of keys equal to T that belong to the set (the lowest-indexed
+// ones).  A final pass over per-warp contiguous segments writes the chosen ids in index order.
 // ------------------------------------------------------------------------------------------------
 constexpr int kTopkThreads = 1024;
+constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kTopkCacheKeys = 16384;
+constexpr int kTopkHistWords = kTopkWarps * 256;
 
-__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *warp_tot, uint32_t *total)
+__device__ __forceinline__ uint32_t block_reduce_minmax(uint32_t v, bool is_max, uint32_t *scratch)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    uint32_t x = v;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
+    for (int o = 16; o > 0; o >>= 1) {
+        const uint32_t y = __shfl_xor_sync(0xffffffffu, v, o);
+        v = is_max ? max(v, y) : min(v, y);
     }
-    if (lane == 31) warp_tot[warp] = x;
+    if (lane == 0) scratch[warp] = v;
     __syncthreads();
     if (warp == 0) {
-        uint32_t t = lane < (int)(blockDim.x >> 5) ? warp_tot[lane] : 0u;
+        v = scratch[lane];
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, t, o);
-            if (lane >= o) t += y;
+        for (int o = 16; o > 0; o >>= 1) {
+            const uint32_t y = __shfl_xor_sync(0xffffffffu, v, o);
+            v = is_max ? max(v, y) : min(v, y);
         }
-        warp_tot[lane] = t;  // inclusive
+        if (lane == 0) scratch[32] = v;
     }
     __syncthreads();
-    const uint32_t before = (warp > 0 ? warp_tot[warp - 1] : 0u) + x - v;
-    *total = warp_tot[(blockDim.x >> 5) - 1];
+    v = scratch[32];
     __syncthreads();
-    return before;
+    return v;
 }
 
 __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const float *__restrict__ scores, int score_stride,
@@ -303,11 +320,13 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const float *__re
                                                                int k, int32_t *__restrict__ out_blocks,
                                                                int32_t *__restrict__ out_count, void *ws)
 {
-    extern __shared__ uint32_t skeys[];
-    __shared__ uint32_t hist[256];
-    __shared__ uint32_t warp_tot[32];
+    extern __shared__ uint32_t tk_smem[];
+    uint32_t *whist = tk_smem;                    // [32 warps][256]
+    uint32_t *skeys = tk_smem + kTopkHistWords;   // cached keys
+    __shared__ uint32_t scratch[40];
+    __shared__ uint32_t wcount[2][kTopkWarps];
     __shared__ uint32_t sel[2];
-    const int b = blockIdx.x, t = threadIdx.x, lane = t & 31;
+    const int b = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int L = seq_len[b];
     int n;
     if (L < 1 || L > max_seq_len) {
@@ -329,70 +348,99 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const float *__re
         return;
     }
     const bool cached = n <= kTopkCacheKeys;
-    if (cached) {
-        for (int i = t; i < n; i += kTopkThreads) skeys[i] = order_key(sc[i]);
-        __syncthreads();
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+    for (int i = t; i < n; i += kTopkThreads) {
+        const uint32_t u = order_key(sc[i]);
+        if (cached) skeys[i] = u;
+        kmin = min(kmin, u);
+        kmax = max(kmax, u);
     }
-    uint32_t prefix = 0, mask = 0;
-    uint32_t remaining = (uint32_t)k;
-    for (int pass = 0; pass < 4; ++pass) {
-        const int shift = 24 - 8 * pass;
-        if (t < 256) hist[t] = 0;
-        __syncthreads();
-        for (int base = 0; base < n; base += kTopkThreads) {
-            const int i = base + t;
-            uint32_t digit = 256;
-            if (i < n) {
+    kmin = block_reduce_minmax(kmin, false, scratch);
+    kmax = block_reduce_minmax(kmax, true, scratch);
+
+    uint32_t prefix = kmax, mask = 0xFFFFFFFFu, remaining = (uint32_t)k;
+    if (kmin != kmax) {
+        int hi = 31 - __clz(kmin ^ kmax);              // highest bit that differs between keys
+        mask = hi == 31 ? 0u : ~((2u << hi) - 1u);
+        prefix = kmax & mask;
+        while (hi >= 0) {
+            const int width = hi + 1 < 8 ? hi + 1 : 8;
+            const int shift = hi + 1 - width;
+            const uint32_t dmask = (1u << width) - 1u;
+            for (int i = t; i < kTopkHistWords; i += kTopkThreads) whist[i] = 0u;
+            __syncthreads();
+            for (int i = t; i < n; i += kTopkThreads) {
                 const uint32_t u = cached ? skeys[i] : order_key(sc[i]);
-                if ((u & mask) == prefix) digit = (u >> shift) & 255u;
+                if ((u & mask) == prefix) atomicAdd(&whist[warp * 256 + ((u >> shift) & dmask)], 1u);
             }
-            const uint32_t peers = __match_any_sync(0xffffffffu, digit);
-            if (digit < 256 && lane == __ffs(peers) - 1) atomicAdd(&hist[digit], (uint32_t)__popc(peers));
-        }
-        __syncthreads();
-        // suffix counts from the top bucket down; the threshold bucket is where they reach `remaining`
-        uint32_t c = 0;
-        if (t < 256) c = hist[255 - t];
-        uint32_t x = c;
+            __syncthreads();
+            // bin totals, then counts from the top bin down; the threshold bin is where they reach
+            // `remaining`
+            uint32_t c = 0;
+            if (t < 256) {
+                const int bin = 255 - t;
+#pragma unroll 8
+                for (int w = 0; w < kTopkWarps; ++w) c += whist[w * 256 + bin];
+            }
+            uint32_t x = c;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += y;
-        }
-        if (t < 256 && lane == 31) warp_tot[t >> 5] = x;
-        __syncthreads();
-        if (t < 256) {
-            uint32_t before = 0;
-            for (int wi = 0; wi < (t >> 5); ++wi) before += warp_tot[wi];
-            const uint32_t incl = before + x;
-            if (incl >= remaining && incl - c < remaining) {
-                sel[0] = 255u - (uint32_t)t;
-                sel[1] = incl - c;
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
             }
+            if (t < 256 && lane == 31) scratch[warp] = x;
+            __syncthreads();
+            if (t < 256) {
+                uint32_t before = 0;
+                for (int wi = 0; wi < warp; ++wi) before += scratch[wi];
+                const uint32_t incl = before + x;
+                if (incl >= remaining && incl - c < remaining) {
+                    sel[0] = 255u - (uint32_t)t;
+                    sel[1] = incl - c;
+                }
+            }
+            __syncthreads();
+            prefix |= sel[0] << shift;
+            mask |= dmask << shift;
+            remaining -= sel[1];
+            hi = shift - 1;
+            __syncthreads();
         }
-        __syncthreads();
-        prefix |= sel[0] << shift;
-        mask |= 255u << shift;
-        remaining -= sel[1];
-        __syncthreads();
     }
     const uint32_t T = prefix, need_eq = remaining;
-    uint32_t gt_run = 0, eq_run = 0;
-    for (int base = 0; base < n; base += kTopkThreads) {
-        const int i = base + t;
+
+    // per-warp contiguous segments: counts, then ordered writes
+    const int seg = (n + kTopkWarps - 1) / kTopkWarps;
+    const int s0 = warp * seg, s1 = min(n, s0 + seg);
+    uint32_t gt_cnt = 0, eq_cnt = 0;
+    for (int base = s0; base < s1; base += 32) {
+        const int i = base + lane;
         uint32_t u = 0;
-        bool gt = false, eq = false;
-        if (i < n) {
-            u = cached ? skeys[i] : order_key(sc[i]);
-            gt = u > T;
-            eq = u == T;
-        }
-        uint32_t tot;
-        const uint32_t ex = block_excl_scan((gt ? 1u : 0u) | (eq ? 0x10000u : 0u), warp_tot, &tot);
-        const uint32_t gt_b = gt_run + (ex & 0xFFFF), eq_b = eq_run + (ex >> 16);
+        if (i < s1) u = cached ? skeys[i] : order_key(sc[i]);
+        gt_cnt += __popc(__ballot_sync(0xffffffffu, i < s1 && u > T));
+        eq_cnt += __popc(__ballot_sync(0xffffffffu, i < s1 && u == T));
+    }
+    if (lane == 0) {
+        wcount[0][warp] = gt_cnt;
+        wcount[1][warp] = eq_cnt;
+    }
+    __syncthreads();
+    uint32_t gt_run = 0, eq_run = 0;
+    for (int wi = 0; wi < warp; ++wi) {
+        gt_run += wcount[0][wi];
+        eq_run += wcount[1][wi];
+    }
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    for (int base = s0; base < s1; base += 32) {
+        const int i = base + lane;
+        uint32_t u = 0;
+        if (i < s1) u = cached ? skeys[i] : order_key(sc[i]);
+        const bool gt = i < s1 && u > T, eq = i < s1 && u == T;
+        const uint32_t bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
+        const uint32_t gt_b = gt_run + __popc(bg & lt_mask), eq_b = eq_run + __popc(be & lt_mask);
         if (gt || (eq && eq_b < need_eq)) out[gt_b + min(eq_b, need_eq)] = ids ? ids[i] : i;
-        gt_run += tot & 0xFFFF;
-        eq_run += tot >> 16;
+        gt_run += __popc(bg);
+        eq_run += __popc(be);
     }
     if (t == 0) out_count[b] = k;
 }
@@ -461,7 +509,7 @@ cudaError_t launch_block_scores_full_or_pool(const uint8_t *keys, int num_pages,
     a.pool = pool;
     a.pool_count = pool_count;
     a.pool_cap = pool_cap;
-    a.items_per_seq = pool ? (pool_cap + kScoreConsumers - 1) / kScoreConsumers
+    a.items_per_seq = pool ? (pool_cap + kScoreWarps - 1) / kScoreWarps
                            : (bt.max_seq_len + kPage - 1) / kPage;
     a.scores = scores;
     a.score_stride = score_stride;
@@ -473,7 +521,8 @@ cudaError_t launch_topk(const float *scores, int score_stride, const int32_t *se
                         const int32_t *pool, const int32_t *pool_count, int pool_cap, int k, int B,
                         int32_t *out_blocks, int32_t *out_count, int max_candidates, void *ws, cudaStream_t st)
 {
-    const size_t smem = (size_t)(max_candidates < kTopkCacheKeys ? max_candidates : kTopkCacheKeys) * 4;
+    const size_t smem =
+        (size_t)kTopkHistWords * 4 + (size_t)(max_candidates < kTopkCacheKeys ? max_candidates : kTopkCacheKeys) * 4;
     cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     topk_kernel<<<B, kTopkThreads, smem, st>>>(scores, score_stride, seq_len, max_seq_len, pool, pool_count, pool_cap,

@@ -59,22 +59,45 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
 }
 
 // Wait for the phase with the given parity to complete.  Returns false (and raises the CTA's abort
-// flag and the workspace status) if the wait runs past kWaitLimitNs or another thread aborted.
+// flag and the workspace status) if the wait runs past kWaitLimitNs or another thread aborted.  The
+// clock and the abort flag are looked at only every 64 polls, so a completed phase is seen within
+// one try_wait.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag, void *ws,
                                           long long where)
 {
     if (mbar_try_wait(bar, parity)) return true;
-    const unsigned long long t0 = global_ns();
-    while (true) {
+    unsigned long long t0 = 0;
+    for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (global_ns() - t0 > kWaitLimitNs) {
-            *abort_flag = 1;
-            report(ws, CSA_ERR_TIMEOUT, where);
-            return false;
+        if ((it & 63u) == 0) {
+            if (*abort_flag) return false;
+            const unsigned long long now = global_ns();
+            if (t0 == 0) {
+                t0 = now;
+            } else if (now - t0 > kWaitLimitNs) {
+                *abort_flag = 1;
+                report(ws, CSA_ERR_TIMEOUT, where);
+                return false;
+            }
         }
     }
 }
+
+// The same wait taken once per warp: lane 0 polls, the outcome is broadcast, so every lane of the
+// warp leaves together (required before warp-collective .aligned instructions).  Call converged.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag, void *ws,
+                                          long long where)
+{
+    int r = 0;
+    if ((threadIdx.x & 31) == 0) r = mbar_wait(bar, parity, abort_flag, ws, where) ? 1 : 0;
+    r = __shfl_sync(0xffffffffu, r, 0);
+    __syncwarp();
+    return r != 0;
+}
+
+// Order this thread's generic-proxy shared-memory accesses with later async-proxy accesses (bulk
+// copies, tensor-core operand reads) of the same memory.
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // 1-D bulk copy global -> this CTA's shared memory, completing `bytes` of transaction on `bar`.
 // Both addresses 16-byte aligned, bytes a multiple of 16.
