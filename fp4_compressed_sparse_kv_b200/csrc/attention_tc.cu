@@ -14,16 +14,22 @@
 // Tile = 128 entries.  Both MMAs put the entries / channels on M = 128 ("swap AB"):
 //   QK:  S^T[128 entries x 64 heads]  = V[128 x 512] . Q^T          (A = V K-major, B = Q K-major)
 //   PV:  O^T[128 ch x 64 heads] (x4)  = V^T[128 ch x 128 entries] . P^T   (A = V^T MN-major, B = P^T MN-major)
-// so TMEM holds S^T in 64 columns and O^T in 256, and one 128-byte-swizzled fp16 copy of the tile in
-// shared memory is read as K-major V by QK and as MN-major V^T by PV.
+//   L :  L^T[128 x 64 heads]          = ones[128 x 128 entries] . P^T      (every row = the column sums of P)
+// so TMEM holds S^T in 64 columns, O^T in 256 and L^T in 64, and one 128-byte-swizzled fp16 copy of
+// the tile in shared memory is read as K-major V by QK and as MN-major V^T by PV.  The all-ones
+// operand is one 128-byte block read through a zero-stride descriptor; summing the same fp16 P on the
+// tensor core keeps the normaliser consistent with the numerator.  Window rows carry their FP8 scale
+// in P (so PV multiplies by it); their sum is corrected by p * (1 - scale) in shared memory.
 //
-// Warp roles (256 threads): warps 0-3 (TMEM lanes 0-127) run the softmax and the epilogue, warp 0
-// owns the TMEM allocation and its lane 0 issues the MMAs between softmax steps (QK of tile t before
-// softmax(t), PV of tile t after it); warps 4-7 load Q once, then dequantise each tile chunk by
-// chunk (64 channels) from raw entries they prefetch into registers.
-// The V buffer is single: chunks of tile t+1 are written as soon as PV(t) has finished the 128-channel
-// M-tile that reads them.  Softmax rescales lazily: O^T in TMEM is rescaled only when a head's
-// running maximum grows by more than 2^8.
+// Warp roles (288 threads).  Warp 8 owns the TMEM allocation and its lane 0 issues every MMA: QK of
+// tile t chunk by chunk as its 64-channel chunks are dequantised, then PV and L of tile t once P is
+// in shared memory.  Group 1 = warps 0-3 (TMEM lanes 0-127) runs the softmax and the epilogue.
+// Group 0 = warps 4-7 loads Q once and writes each tile's entry metadata.  Both groups dequantise:
+// thread e of a group takes tile row e and the group's four 64-channel chunks (0, 1, 4, 5 for group
+// 0; 2, 3, 6, 7 for group 1) from raw entries prefetched into registers a tile ahead.  The V buffer
+// is single; the chunks of tile t+1 are written as soon as PV(t) has finished the M-tile reading
+// them, so dequantisation and the QK of tile t+1 overlap the end of PV(t).  Softmax rescales lazily:
+// O^T and L^T are rescaled in TMEM only when a head's running maximum grows by more than 2^8.
 #include "attention_common.cuh"
 #include "pipeline.cuh"
 #include "tcgen05.cuh"
@@ -34,16 +40,18 @@ constexpr int kTcHeads = 64;
 constexpr int kTcRows = 128;
 constexpr int kTcUnits = kTcRows / kAttnUnit;
 constexpr int kTcChunks = kLatent / 64;
-constexpr int kTcThreads = 256;   // 4 softmax/MMA warps, 4 dequant warps
+constexpr int kTcThreads = 288;   // 4 softmax warps, 4 dequant warps, 1 MMA warp
 constexpr uint32_t kVChunk = kTcRows * 128;   // 16 KB: 128 rows x 64 fp16
 constexpr uint32_t kQChunk = kTcHeads * 128;  // 8 KB: 64 rows x 64 fp16
 constexpr uint32_t kOffV = 0;
 constexpr uint32_t kOffQ = kOffV + kTcChunks * kVChunk;
 constexpr uint32_t kOffP = kOffQ + kTcChunks * kQChunk;
-constexpr uint32_t kOffMisc = kOffP + kTcRows * 128;
+constexpr uint32_t kOffOnes = kOffP + kTcRows * 128;   // 128 B of fp16 ones
+constexpr uint32_t kOffMisc = kOffOnes + 1024;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;
 constexpr uint32_t kColO = 64;
+constexpr uint32_t kColL = 320;
 constexpr float kLazy = 8.f;      // log2-domain growth of a head maximum tolerated without rescaling
 constexpr float kPOffset = 7.f;   // p = exp2(z - m + 7) <= 2^15 keeps small p out of fp16 subnormals
 constexpr float kLog2e = 1.4426950408889634f;
@@ -53,14 +61,13 @@ struct TcMisc {
     uint64_t s_full, p_full, q_ready, o_done, final_bar;
     uint64_t v_ready[kTcChunks];
     uint64_t v_free[kTcChunks / 2];
-    uint64_t sm_bar;            // softmax warpgroup sync (bounded, unlike a named barrier)
     uint32_t tmem_base;
     int abort_flag;
-    int vote[4];
     float vmeta[2][kTcRows];    // per entry: -1 masked, else its value scale (1 for FP4, window scale)
     float zscale[kTcHeads];     // tau * 2^-k_h * log2(e)
     float m[kTcHeads];          // running max, log2 domain
     float alpha[kTcHeads];
+    float lcorr[kTcHeads];      // sum over window rows of p * (1 - scale): their P carries the scale
     float red[4][kTcHeads];
 };
 
@@ -68,6 +75,7 @@ constexpr size_t kTcSmem = kOffMisc + sizeof(TcMisc) + 1024;
 
 constexpr uint32_t kIdescQK = umma_idesc_f16(128, kTcHeads, false, false);
 constexpr uint32_t kIdescPV = umma_idesc_f16(128, kTcHeads, true, true);
+constexpr uint32_t kIdescL = umma_idesc_f16(128, kTcHeads, false, true);
 
 __device__ __forceinline__ uint32_t swz(uint32_t row, uint32_t unit) { return row * 128u + ((unit ^ (row & 7u)) << 4); }
 
@@ -85,6 +93,160 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi)
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
+// Softmax warpgroup barriers (named barrier 1, the 128 threads of warps 0-3).  Every thread of the
+// group executes each of them once per tile, also after a failed wait, so none can be left waiting.
+__device__ __forceinline__ bool group_and(bool v)
+{
+    int r;
+    asm volatile("{\n.reg .pred p, q;\nsetp.ne.b32 q, %1, 0;\nbar.red.and.pred p, 1, 128, q;\nselp.b32 %0, 1, 0, p;\n}"
+                 : "=r"(r)
+                 : "r"((int)v)
+                 : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ bool group_or(bool v)
+{
+    int r;
+    asm volatile("{\n.reg .pred p, q;\nsetp.ne.b32 q, %1, 0;\nbar.red.or.pred p, 1, 128, q;\nselp.b32 %0, 1, 0, p;\n}"
+                 : "=r"(r)
+                 : "r"((int)v)
+                 : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ void group_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// One thread's share of a tile's dequantisation: entry e (tile row) and the four 64-channel chunks of
+// its thread group (group 0: chunks 0, 1, 4, 5; group 1: chunks 2, 3, 6, 7), raw bytes prefetched
+// into registers.
+struct TileRows {
+    EntryRef r;
+    bool valid;
+    uint4 code[8];     // code bytes of the group's chunks: 64 B at 64*g, 64 B at 128 + 64*g
+    uint2 scl[2];      // their scale words
+
+    __device__ __forceinline__ void load(const AttnArgs &a, const SeqView &sv, int u_begin, int u_end, int t, int e,
+                                         int g)
+    {
+        const int u = u_begin + t * kTcUnits + e / kAttnUnit, j = e % kAttnUnit;
+        valid = u < u_end && entry_ref(a, sv, u, j, r);
+        if (valid && !r.swa) {
+            const uint4 *cp = reinterpret_cast<const uint4 *>(r.p);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                code[q] = cp[4 * g + q];
+                code[4 + q] = cp[8 + 4 * g + q];
+            }
+            const uint2 *sp = reinterpret_cast<const uint2 *>(r.sc);
+            scl[0] = sp[g];
+            scl[1] = sp[2 + g];
+        }
+    }
+
+    // Chunk slot cs (0..3) of this group: channels 64c .. 64c+63, c = 2g + (cs & 1) + 4 (cs >> 1).
+    __device__ __forceinline__ void write(uint8_t *V, int e, int c, int cs) const
+    {
+        uint4 out[8];
+        if (!valid) {
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) out[jj] = make_uint4(0u, 0u, 0u, 0u);
+        } else if (!r.swa) {
+            const uint32_t sw = (cs & 1) ? scl[cs >> 1].y : scl[cs >> 1].x;
+#pragma unroll
+            for (int gg = 0; gg < 4; ++gg) {
+                const uint32_t sh = e4m3x2_to_f16x2((uint16_t)((sw >> (8 * gg)) & 0xFF));
+                const uint32_t s2 = (sh & 0xFFFFu) | (sh << 16);
+                const uint4 cw = code[2 * cs + (gg >> 1)];
+                const uint32_t w0 = (gg & 1) ? cw.z : cw.x, w1 = (gg & 1) ? cw.w : cw.y;
+                uint32_t v[8];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    v[q] = hmul2_u32(e2m1x2_to_f16x2((uint8_t)(w0 >> (8 * q))), s2);
+                    v[4 + q] = hmul2_u32(e2m1x2_to_f16x2((uint8_t)(w1 >> (8 * q))), s2);
+                }
+                out[2 * gg] = make_uint4(v[0], v[1], v[2], v[3]);
+                out[2 * gg + 1] = make_uint4(v[4], v[5], v[6], v[7]);
+            }
+        } else {
+            // window entry: 64 E4M3 values, exact in fp16; its scale is applied in the softmax
+            const uint4 *src = reinterpret_cast<const uint4 *>(r.p + 64 * c);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint4 w = src[q];
+                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+                uint32_t v[8];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    v[2 * k] = e4m3x2_to_f16x2((uint16_t)(ww[k] & 0xFFFF));
+                    v[2 * k + 1] = e4m3x2_to_f16x2((uint16_t)(ww[k] >> 16));
+                }
+                out[2 * q] = make_uint4(v[0], v[1], v[2], v[3]);
+                out[2 * q + 1] = make_uint4(v[4], v[5], v[6], v[7]);
+            }
+        }
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) *reinterpret_cast<uint4 *>(V + c * kVChunk + swz((uint32_t)e, (uint32_t)jj)) = out[jj];
+    }
+};
+
+// Dequantise this group's four chunks of tile t into V (waiting for PV(t-1) to release each pair).
+__device__ __forceinline__ bool dequant_group(TcMisc &ms, uint8_t *V, const TileRows &rows, const AttnArgs &a, int t,
+                                              int e, int g)
+{
+    bool ok = true;
+#pragma unroll
+    for (int cs = 0; cs < 4; ++cs) {
+        const int c = 2 * g + (cs & 1) + 4 * (cs >> 1);
+        if (t > 0 && (cs & 1) == 0) ok = ok && warp_wait(&ms.v_free[c >> 1], (t - 1) & 1, &ms.abort_flag, a.ws, 5);
+        if (ok) rows.write(V, e, c, cs);
+        fence_async_smem();
+        mbar_arrive(&ms.v_ready[c]);
+    }
+    return ok;
+}
+
+// Q of heads h0..h0+63 into shared memory as fp16, 128B-swizzled K-major, each head scaled by a power
+// of two 2^k_h that puts its largest |q| in [2^13, 2^14); the softmax undoes it through zscale.
+// Thread t of the 256 dequantising threads converts a quarter row (128 channels) of head t/4.
+__device__ __forceinline__ void load_q(const AttnArgs &a, TcMisc &ms, uint8_t *Q, int b, int h0, int t)
+{
+    const int h = t >> 2, quarter = t & 3;
+    const uint4 *qrow = reinterpret_cast<const uint4 *>(a.q + ((size_t)b * a.H + h0 + h) * kLatent + quarter * 128);
+    uint4 qw[16];
+#pragma unroll
+    for (int c = 0; c < 16; ++c) qw[c] = qrow[c];
+    float amax = 0.f;
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+        const uint32_t ww[4] = {qw[c].x, qw[c].y, qw[c].z, qw[c].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(ww[k])), fabsf(bf16_hi(ww[k]))));
+    }
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    int k = 0;
+    if (amax > 0.f) {
+        const int ex = (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127;
+        k = 13 - ex;
+        k = k < -60 ? -60 : (k > 60 ? 60 : k);
+    }
+    const float sc = exp2f((float)k);
+    if (quarter == 0) ms.zscale[h] = a.sm_scale * exp2f((float)-k) * kLog2e;
+#pragma unroll
+    for (int c = 0; c < 16; ++c) {
+        uint4 o;
+        o.x = pack_f16x2(bf16_lo(qw[c].x) * sc, bf16_hi(qw[c].x) * sc);
+        o.y = pack_f16x2(bf16_lo(qw[c].y) * sc, bf16_hi(qw[c].y) * sc);
+        o.z = pack_f16x2(bf16_lo(qw[c].z) * sc, bf16_hi(qw[c].z) * sc);
+        o.w = pack_f16x2(bf16_lo(qw[c].w) * sc, bf16_hi(qw[c].w) * sc);
+        const int ch = quarter * 128 + 8 * c;
+        *reinterpret_cast<uint4 *>(Q + (ch >> 6) * kQChunk + swz(h, (ch & 63) >> 3)) = o;
+    }
+    fence_async_smem();
+    mbar_arrive(&ms.q_ready);
+}
+
 __global__ void __launch_bounds__(kTcThreads, 1) attn_split_tc_kernel(AttnArgs a, int head_groups)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -92,6 +254,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_split_tc_kernel(AttnArgs a
     uint8_t *V = base + kOffV;
     uint8_t *Q = base + kOffQ;
     uint8_t *P = base + kOffP;
+    uint8_t *ONES = base + kOffOnes;
     TcMisc &ms = *reinterpret_cast<TcMisc *>(base + kOffMisc);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -107,326 +270,251 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_split_tc_kernel(AttnArgs a
     if (threadIdx.x == 0) {
         mbar_init(&ms.s_full, 1);
         mbar_init(&ms.p_full, 128);
-        mbar_init(&ms.q_ready, 128);
+        mbar_init(&ms.q_ready, 256);
         mbar_init(&ms.o_done, 1);
         mbar_init(&ms.final_bar, 1);
         for (int c = 0; c < kTcChunks; ++c) mbar_init(&ms.v_ready[c], 128);
         for (int c = 0; c < kTcChunks / 2; ++c) mbar_init(&ms.v_free[c], 1);
-        mbar_init(&ms.sm_bar, 128);
         ms.abort_flag = 0;
         fence_mbar_init();
     }
-    if (threadIdx.x < kTcHeads) ms.m[threadIdx.x] = -INFINITY;
-    if (warp == 0 && ntiles > 0) {
+    if (threadIdx.x < kTcHeads) {
+        ms.m[threadIdx.x] = -INFINITY;
+        ms.lcorr[threadIdx.x] = 0.f;
+    }
+    if (threadIdx.x < 32) reinterpret_cast<uint32_t *>(ONES)[threadIdx.x] = 0x3C003C00u;   // fp16 1.0 pairs
+    if (warp == 8 && ntiles > 0) {
         tc_alloc(smem_addr(&ms.tmem_base), kTmemCols);
         tc_relinquish();
     }
+    fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ms.tmem_base;
 
-    if (warp >= 4) {
-        // ------------------------------- Q load, then dequantisation ------------------------
-        const int i = threadIdx.x - 128;   // 0..127
-        {
-            // Q: thread i converts half a head row (256 channels); per-head power-of-two scale
-            const int h = i >> 1, half = i & 1;
-            const uint16_t *qrow = a.q + ((size_t)b * a.H + h0 + h) * kLatent + half * 256;
-            float amax = 0.f;
-            for (int c = 0; c < 256; c += 8) {
-                const uint4 w = *reinterpret_cast<const uint4 *>(qrow + c);
-                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                for (int k = 0; k < 4; ++k) amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(ww[k])), fabsf(bf16_hi(ww[k]))));
-            }
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-            int k = 0;
-            if (amax > 0.f) {
-                const int e = (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127;
-                k = 13 - e;
-                k = k < -60 ? -60 : (k > 60 ? 60 : k);
-            }
-            const float sc = exp2f((float)k);
-            if (half == 0) ms.zscale[h] = a.sm_scale * exp2f((float)-k) * kLog2e;
-            for (int c = 0; c < 256; c += 8) {
-                const uint4 w = *reinterpret_cast<const uint4 *>(qrow + c);
-                uint4 o;
-                o.x = pack_f16x2(bf16_lo(w.x) * sc, bf16_hi(w.x) * sc);
-                o.y = pack_f16x2(bf16_lo(w.y) * sc, bf16_hi(w.y) * sc);
-                o.z = pack_f16x2(bf16_lo(w.z) * sc, bf16_hi(w.z) * sc);
-                o.w = pack_f16x2(bf16_lo(w.w) * sc, bf16_hi(w.w) * sc);
-                const int ch = half * 256 + c;
-                *reinterpret_cast<uint4 *>(Q + (ch >> 6) * kQChunk + swz(h, (ch & 63) >> 3)) = o;
-            }
-            fence_async_smem();
-            mbar_arrive(&ms.q_ready);
+    if (ntiles == 0) {
+        // empty split: a neutral partial
+        if (warp < 4) {
+            float *po = a.part_o + (((size_t)b * a.splits + s) * a.H + h0) * kLatent;
+            for (int h = 0; h < kTcHeads; ++h)
+                for (int c = threadIdx.x; c < kLatent; c += 128) po[(size_t)h * kLatent + c] = 0.f;
+            if (threadIdx.x < kTcHeads)
+                reinterpret_cast<float2 *>(a.part_ml)[((size_t)b * a.splits + s) * a.H + h0 + threadIdx.x] =
+                    make_float2(-INFINITY, 0.f);
         }
-        bool ok = true;
-        for (int t = 0; ok && t < ntiles; ++t) {
-            const int u = u_begin + t * kTcUnits + i / kAttnUnit, j = i % kAttnUnit;
-            EntryRef r;
-            const bool valid = u < u_end && entry_ref(a, sv, u, j, r);
-            uint4 craw[16];
-            uint4 sraw[2];
-            if (valid && !r.swa) {
-#pragma unroll
-                for (int q = 0; q < 16; ++q) craw[q] = reinterpret_cast<const uint4 *>(r.p)[q];
-                sraw[0] = reinterpret_cast<const uint4 *>(r.sc)[0];
-                sraw[1] = reinterpret_cast<const uint4 *>(r.sc)[1];
-            }
-            ms.vmeta[t & 1][i] = valid ? (r.swa ? r.fscale : 1.f) : -1.f;
-#pragma unroll
-            for (int c = 0; c < kTcChunks; ++c) {
-                if (t > 0 && (c & 1) == 0) {
-                    ok = warp_wait(&ms.v_free[c >> 1], (t - 1) & 1, &ms.abort_flag, a.ws, 5);
-                    if (!ok) break;
-                }
-                uint4 out[8];
-                if (!valid) {
-#pragma unroll
-                    for (int jj = 0; jj < 8; ++jj) out[jj] = make_uint4(0u, 0u, 0u, 0u);
-                } else if (!r.swa) {
-                    // channels 64c .. 64c+63: code bytes 32c .. 32c+31, scale groups 4c .. 4c+3
-                    const uint32_t sw = (c < 4) ? (&sraw[0].x)[c] : (&sraw[1].x)[c - 4];
-#pragma unroll
-                    for (int g = 0; g < 4; ++g) {
-                        const uint32_t sh = e4m3x2_to_f16x2((uint16_t)((sw >> (8 * g)) & 0xFF));
-                        const uint32_t s2 = (sh & 0xFFFFu) | (sh << 16);
-                        const uint4 cw = craw[2 * c + (g >> 1)];
-                        const uint32_t w0 = (g & 1) ? cw.z : cw.x, w1 = (g & 1) ? cw.w : cw.y;
-                        uint32_t v[8];
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            v[q] = hmul2_u32(e2m1x2_to_f16x2((uint8_t)(w0 >> (8 * q))), s2);
-                            v[4 + q] = hmul2_u32(e2m1x2_to_f16x2((uint8_t)(w1 >> (8 * q))), s2);
-                        }
-                        out[2 * g] = make_uint4(v[0], v[1], v[2], v[3]);
-                        out[2 * g + 1] = make_uint4(v[4], v[5], v[6], v[7]);
-                    }
-                } else {
-                    // window entry: 64 E4M3 values, exact in fp16; its scale is applied in the softmax
-                    const uint4 *src = reinterpret_cast<const uint4 *>(r.p + 64 * c);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint4 w = src[q];
-                        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-                        uint32_t v[8];
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            v[2 * k] = e4m3x2_to_f16x2((uint16_t)(ww[k] & 0xFFFF));
-                            v[2 * k + 1] = e4m3x2_to_f16x2((uint16_t)(ww[k] >> 16));
-                        }
-                        out[2 * q] = make_uint4(v[0], v[1], v[2], v[3]);
-                        out[2 * q + 1] = make_uint4(v[4], v[5], v[6], v[7]);
-                    }
-                }
-#pragma unroll
-                for (int jj = 0; jj < 8; ++jj)
-                    *reinterpret_cast<uint4 *>(V + c * kVChunk + swz((uint32_t)i, (uint32_t)jj)) = out[jj];
-                fence_async_smem();
-                mbar_arrive(&ms.v_ready[c]);
-            }
-        }
-    } else if (warp < 4) {
-        // ------------------------------- softmax + epilogue -------------------------------
-        const int e = threadIdx.x;              // TMEM lane = tile row (entry) / channel in epilogue
-        const int wq = warp & 3;
-        const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
-        float lsum[kTcHeads];
-#pragma unroll
-        for (int h = 0; h < kTcHeads; ++h) lsum[h] = 0.f;
-        bool ok = ntiles > 0;
-        uint32_t sync_phase = 0;
-        // all 128 softmax threads arrive, then wait with a time limit; false on timeout or abort
-        auto sync128 = [&]() -> bool {
-            mbar_arrive(&ms.sm_bar);
-            const bool r = warp_wait(&ms.sm_bar, sync_phase & 1, &ms.abort_flag, a.ws, 9);
-            ++sync_phase;
-            return r;
-        };
-        const uint32_t sV = smem_addr(V), sQ = smem_addr(Q), sP = smem_addr(P);
-        const bool issuer = warp == 0 && lane == 0;
-        // Q and the per-head score scales are in shared memory (written by the dequant warps)
-        if (ntiles > 0) {
-            ok = warp_wait(&ms.q_ready, 0, &ms.abort_flag, a.ws, 1);
+        return;
+    }
+
+    if (warp == 8) {
+        // ------------------------------- MMA issuer -------------------------------
+        if (lane == 0) {
+            const uint32_t sV = smem_addr(V), sQ = smem_addr(Q), sP = smem_addr(P), sOnes = smem_addr(ONES);
+            const uint64_t ones_desc = umma_sdesc_noswz(sOnes, 0, 0);
+            bool ok = mbar_wait(&ms.q_ready, 0, &ms.abort_flag, a.ws, 1);
             tc_fence_after();
-        }
-        for (int t = 0; ok && t < ntiles; ++t) {
-            const uint32_t ph = t & 1;
-            if (warp == 0) {
-                // QK of tile t, chunk by chunk as the dequantisation lands
-                int iok = 1;
-                if (issuer) {
-                    for (int c = 0; c < kTcChunks; ++c) {
-                        if (!mbar_wait(&ms.v_ready[c], ph, &ms.abort_flag, a.ws, 2)) {
-                            iok = 0;
-                            break;
-                        }
-                        tc_fence_after();
+            for (int t = 0; ok && t < ntiles; ++t) {
+                const uint32_t ph = t & 1;
+                for (int c = 0; c < kTcChunks; ++c) {
+                    if (!(ok = mbar_wait(&ms.v_ready[c], ph, &ms.abort_flag, a.ws, 2))) break;
+                    tc_fence_after();
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            const uint64_t ad = umma_sdesc_sw128(sV + c * kVChunk + kk * 32, 16, 1024);
-                            const uint64_t bd = umma_sdesc_sw128(sQ + c * kQChunk + kk * 32, 16, 1024);
-                            tc_mma_f16(tmem + kColS, ad, bd, kIdescQK, (c | kk) != 0);
-                        }
-                    }
-                    if (iok) tc_commit(smem_addr(&ms.s_full));
-                }
-                if (!__shfl_sync(0xffffffffu, iok, 0)) {
-                    ok = false;
-                    break;
-                }
-            }
-            ok = warp_wait(&ms.s_full, ph, &ms.abort_flag, a.ws, 6) &&
-                 warp_wait(&ms.v_ready[kTcChunks - 1], ph, &ms.abort_flag, a.ws, 7);
-            if (!ok) break;
-            tc_fence_after();
-            float z[kTcHeads];
-            tc_ld32(tl + kColS, z);
-            tc_ld32(tl + kColS + 32, z + 32);
-            tc_wait_ld();
-            const float em = ms.vmeta[ph][e];
-            const bool valid = em >= 0.f;
-            bool need = false;
-#pragma unroll
-            for (int h = 0; h < kTcHeads; ++h) {
-                z[h] = valid ? z[h] * (em * ms.zscale[h]) : -INFINITY;
-                need |= z[h] > ms.m[h] + kLazy;
-            }
-            const bool wneed = __any_sync(0xffffffffu, need);
-            if (lane == 0) ms.vote[wq] = wneed ? 1 : 0;
-            if (!(ok = sync128())) break;
-            const bool rescale = ms.vote[0] | ms.vote[1] | ms.vote[2] | ms.vote[3];
-            if (rescale) {
-#pragma unroll
-                for (int h = 0; h < kTcHeads; ++h) {
-                    float v = z[h];
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-                    if (lane == 0) ms.red[wq][h] = v;
-                }
-                if (!(ok = sync128())) break;
-                if (e < kTcHeads) {
-                    const float mt = fmaxf(fmaxf(ms.red[0][e], ms.red[1][e]), fmaxf(ms.red[2][e], ms.red[3][e]));
-                    const float mo = ms.m[e];
-                    const float mn = fmaxf(mo, mt);
-                    ms.alpha[e] = (mo == -INFINITY) ? 0.f : exp2f(mo - mn);
-                    ms.m[e] = mn;
-                }
-                if (!(ok = sync128())) break;
-#pragma unroll
-                for (int h = 0; h < kTcHeads; ++h) lsum[h] *= ms.alpha[h];
-                if (t > 0) {
-                    for (int m = 0; m < 4; ++m) {
-#pragma unroll
-                        for (int half = 0; half < 2; ++half) {
-                            float o[32];
-                            const uint32_t col = kColO + 64 * m + 32 * half;
-                            tc_ld32(tl + col, o);
-                            tc_wait_ld();
-#pragma unroll
-                            for (int q = 0; q < 32; ++q) o[q] *= ms.alpha[32 * half + q];
-                            tc_st32(tl + col, o);
-                        }
-                    }
-                    tc_wait_st();
-                }
-            }
-            const float pv_scale = valid ? em : 0.f;
-            uint32_t pk[kTcHeads / 2];
-#pragma unroll
-            for (int h = 0; h < kTcHeads; h += 2) {
-                const float p0 = exp2f(z[h] - ms.m[h] + kPOffset);
-                const float p1 = exp2f(z[h + 1] - ms.m[h + 1] + kPOffset);
-                lsum[h] += p0;
-                lsum[h + 1] += p1;
-                pk[h / 2] = pack_f16x2(p0 * pv_scale, p1 * pv_scale);
-            }
-#pragma unroll
-            for (int jj = 0; jj < 8; ++jj)
-                *reinterpret_cast<uint4 *>(P + swz((uint32_t)e, (uint32_t)jj)) =
-                    make_uint4(pk[4 * jj], pk[4 * jj + 1], pk[4 * jj + 2], pk[4 * jj + 3]);
-            fence_async_smem();
-            tc_fence_before();
-            mbar_arrive(&ms.p_full);
-            if (warp == 0) {
-                // PV of tile t once all 128 rows of P are in shared memory
-                int iok = 1;
-                if (issuer) {
-                    if (!mbar_wait(&ms.p_full, ph, &ms.abort_flag, a.ws, 3)) {
-                        iok = 0;
-                    } else {
-                        tc_fence_after();
-                        for (int m = 0; m < 4; ++m) {
-#pragma unroll
-                            for (int kk = 0; kk < kTcRows / 16; ++kk) {
-                                const uint64_t ad = umma_sdesc_sw128(sV + 2 * m * kVChunk + kk * 2048, kVChunk, 1024);
-                                const uint64_t bd = umma_sdesc_sw128(sP + kk * 2048, kVChunk, 1024);
-                                tc_mma_f16(tmem + kColO + 64 * m, ad, bd, kIdescPV, (t > 0 || kk > 0) ? 1u : 0u);
-                            }
-                            tc_commit(smem_addr(&ms.v_free[m]));
-                        }
-                        if (t == ntiles - 1) tc_commit(smem_addr(&ms.o_done));
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t ad = umma_sdesc_sw128(sV + c * kVChunk + kk * 32, 16, 1024);
+                        const uint64_t bd = umma_sdesc_sw128(sQ + c * kQChunk + kk * 32, 16, 1024);
+                        tc_mma_f16(tmem + kColS, ad, bd, kIdescQK, (c | kk) != 0);
                     }
                 }
-                if (!__shfl_sync(0xffffffffu, iok, 0)) {
-                    ok = false;
-                    break;
+                if (!ok) break;
+                tc_commit(smem_addr(&ms.s_full));
+                if (!(ok = mbar_wait(&ms.p_full, ph, &ms.abort_flag, a.ws, 3))) break;
+                tc_fence_after();
+                for (int m = 0; m < 4; ++m) {
+#pragma unroll
+                    for (int kk = 0; kk < kTcRows / 16; ++kk) {
+                        const uint64_t ad = umma_sdesc_sw128(sV + 2 * m * kVChunk + kk * 2048, kVChunk, 1024);
+                        const uint64_t bd = umma_sdesc_sw128(sP + kk * 2048, kVChunk, 1024);
+                        tc_mma_f16(tmem + kColO + 64 * m, ad, bd, kIdescPV, (t > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    tc_commit(smem_addr(&ms.v_free[m]));
                 }
+#pragma unroll
+                for (int kk = 0; kk < kTcRows / 16; ++kk) {
+                    const uint64_t bd = umma_sdesc_sw128(sP + kk * 2048, kVChunk, 1024);
+                    tc_mma_f16(tmem + kColL, ones_desc, bd, kIdescL, (t > 0 || kk > 0) ? 1u : 0u);
+                }
+                if (t == ntiles - 1) tc_commit(smem_addr(&ms.o_done));
             }
-        }
-        if (issuer && ntiles > 0) {
             // every MMA this thread issued has completed before TMEM is released
             tc_commit(smem_addr(&ms.final_bar));
             volatile int no_abort = 0;
             mbar_wait(&ms.final_bar, 0, &no_abort, a.ws, 4);
         }
         __syncwarp();
+    } else if (warp >= 4) {
+        // ------------------------- group 0: Q load, tile metadata, chunks 0, 1, 4, 5 -------------------
+        const int i = threadIdx.x - 128;   // 0..127
+        TileRows rows;
+        rows.load(a, sv, u_begin, u_end, 0, i, 0);
+        load_q(a, ms, Q, b, h0, threadIdx.x);
+        bool ok = true;
+        for (int t = 0; ok && t < ntiles; ++t) {
+            if (t > 0) rows.load(a, sv, u_begin, u_end, t, i, 0);
+            ms.vmeta[t & 1][i] = rows.valid ? (rows.r.swa ? rows.r.fscale : 1.f) : -1.f;
+            ok = dequant_group(ms, V, rows, a, t, i, 0);
+        }
+    } else {
+        // ------------------------- group 1: softmax, chunks 2, 3, 6, 7, epilogue ----------------------
+        const int e = threadIdx.x;          // TMEM lane = tile row (entry); channel in the epilogue
+        const int wq = warp;
+        const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
+        TileRows rows;
+        rows.load(a, sv, u_begin, u_end, 0, e, 1);
+        load_q(a, ms, Q, b, h0, threadIdx.x);
+        bool ok = dequant_group(ms, V, rows, a, 0, e, 1);
+        // the per-head score scales (written by group 0 before q_ready)
+        ok = warp_wait(&ms.q_ready, 0, &ms.abort_flag, a.ws, 1) && ok;
+        ok = group_and(ok);
+        for (int t = 0; ok && t < ntiles; ++t) {
+            const uint32_t ph = t & 1;
+            bool tok = warp_wait(&ms.s_full, ph, &ms.abort_flag, a.ws, 6) &&
+                       warp_wait(&ms.v_ready[0], ph, &ms.abort_flag, a.ws, 7);
+            if (!(ok = group_and(tok))) break;
+            tc_fence_after();
+            const float em = ms.vmeta[ph][e];
+            const bool valid = em >= 0.f;
+            // scores of heads 32*half .. 32*half+31, scaled to the log2 domain (masked rows: -inf)
+            auto load_z = [&](int half, float *zt) {
+                tc_ld32(tl + kColS + 32 * half, zt);
+                tc_wait_ld();
+#pragma unroll
+                for (int q = 0; q < 32; ++q) zt[q] = valid ? zt[q] * (em * ms.zscale[32 * half + q]) : -INFINITY;
+            };
+            bool need = false;
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                float zt[32];
+                load_z(half, zt);
+#pragma unroll
+                for (int q = 0; q < 32; ++q) need |= zt[q] > ms.m[32 * half + q] + kLazy;
+            }
+            if (group_or(need)) {
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+                    float zt[32];
+                    load_z(half, zt);
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) {
+                        float v = zt[q];
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+                        if (lane == 0) ms.red[wq][32 * half + q] = v;
+                    }
+                }
+                group_sync();
+                if (e < kTcHeads) {
+                    const float mt = fmaxf(fmaxf(ms.red[0][e], ms.red[1][e]), fmaxf(ms.red[2][e], ms.red[3][e]));
+                    const float mo = ms.m[e];
+                    const float mn = fmaxf(mo, mt);
+                    const float al = (mo == -INFINITY) ? 0.f : exp2f(mo - mn);
+                    ms.alpha[e] = al;
+                    ms.m[e] = mn;
+                    ms.lcorr[e] *= al;
+                }
+                group_sync();
+                if (t > 0) {
+                    // O^T (4 M-tiles) and L^T columns, per-head factors
+#pragma unroll 1
+                    for (int m = 0; m < 10; ++m) {
+                        float o[32];
+                        const uint32_t col = kColO + 32 * m;
+                        tc_ld32(tl + col, o);
+                        tc_wait_ld();
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) o[q] *= ms.alpha[32 * (m & 1) + q];
+                        tc_st32(tl + col, o);
+                    }
+                    tc_wait_st();
+                }
+            }
+            const float pv_scale = valid ? em : 0.f;
+            const bool scaled_row = valid && em != 1.f;   // a window entry
+            const bool warp_scaled = __any_sync(0xffffffffu, scaled_row);
+            const float cf = scaled_row ? 1.f - em : 0.f;
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                float zt[32];
+                load_z(half, zt);
+                uint32_t pk[16];
+#pragma unroll
+                for (int q = 0; q < 32; q += 2) {
+                    const float p0 = exp2f(zt[q] - ms.m[32 * half + q] + kPOffset);
+                    const float p1 = exp2f(zt[q + 1] - ms.m[32 * half + q + 1] + kPOffset);
+                    pk[q / 2] = pack_f16x2(p0 * pv_scale, p1 * pv_scale);
+                    zt[q] = p0 * cf;          // reused: the window-row correction of the sums
+                    zt[q + 1] = p1 * cf;
+                }
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj)
+                    *reinterpret_cast<uint4 *>(P + swz((uint32_t)e, (uint32_t)(4 * half + jj))) =
+                        make_uint4(pk[4 * jj], pk[4 * jj + 1], pk[4 * jj + 2], pk[4 * jj + 3]);
+                if (warp_scaled) {
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) {
+                        float v = zt[q];
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                        if (lane == 0) atomicAdd(&ms.lcorr[32 * half + q], v);
+                    }
+                }
+            }
+            fence_async_smem();
+            tc_fence_before();
+            mbar_arrive(&ms.p_full);
+            // this group's chunks of the next tile, as PV(t) releases them
+            if (t + 1 < ntiles) {
+                rows.load(a, sv, u_begin, u_end, t + 1, e, 1);
+                dequant_group(ms, V, rows, a, t + 1, e, 1);
+            }
+        }
         // ---- epilogue: partial (o, m, l) of this split
         float *po = a.part_o + (((size_t)b * a.splits + s) * a.H + h0) * kLatent;
         float2 *pml = reinterpret_cast<float2 *>(a.part_ml) + ((size_t)b * a.splits + s) * a.H + h0;
-        if (ntiles == 0) {
-            for (int h = 0; h < kTcHeads; ++h) {
-                po[(size_t)h * kLatent + e] = 0.f;
-                po[(size_t)h * kLatent + 128 + e] = 0.f;
-                po[(size_t)h * kLatent + 256 + e] = 0.f;
-                po[(size_t)h * kLatent + 384 + e] = 0.f;
-            }
-            if (e < kTcHeads) pml[e] = make_float2(-INFINITY, 0.f);
-        } else if (ok) {
-            ok = warp_wait(&ms.o_done, 0, &ms.abort_flag, a.ws, 8);
+        bool eok = ok && warp_wait(&ms.o_done, 0, &ms.abort_flag, a.ws, 8);
+        eok = group_and(eok);
+        if (eok) {
             tc_fence_after();
+            for (int m = 0; m < 4; ++m) {
 #pragma unroll
-            for (int h = 0; h < kTcHeads; ++h) {
-                float v = lsum[h];
+                for (int half = 0; half < 2; ++half) {
+                    float o[32];
+                    tc_ld32(tl + kColO + 64 * m + 32 * half, o);
+                    tc_wait_ld();
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                if (lane == 0) ms.red[wq][h] = v;
+                    for (int q = 0; q < 32; ++q) po[(size_t)(32 * half + q) * kLatent + 128 * m + e] = o[q];
+                }
             }
-            ok = ok && sync128();
-            if (ok) {
-                for (int m = 0; m < 4; ++m) {
+            if (warp == 0) {
+                // every row of L^T holds the sums; lane 0's row is shared through shared memory
+                float l[32];
 #pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        float o[32];
-                        tc_ld32(tl + kColO + 64 * m + 32 * half, o);
-                        tc_wait_ld();
+                for (int half = 0; half < 2; ++half) {
+                    tc_ld32(tl + kColL + 32 * half, l);
+                    tc_wait_ld();
+                    if (lane == 0) {
 #pragma unroll
-                        for (int q = 0; q < 32; ++q) po[(size_t)(32 * half + q) * kLatent + 128 * m + e] = o[q];
+                        for (int q = 0; q < 32; ++q) ms.red[0][32 * half + q] = l[q];
                     }
                 }
-                if (e < kTcHeads) {
-                    const float l = ms.red[0][e] + ms.red[1][e] + ms.red[2][e] + ms.red[3][e];
-                    pml[e] = make_float2((ms.m[e] - kPOffset) * kLn2, l);
-                }
             }
+            group_sync();
+            if (e < kTcHeads) pml[e] = make_float2((ms.m[e] - kPOffset) * kLn2, ms.red[0][e] + ms.lcorr[e]);
         }
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 0 && ntiles > 0) tc_dealloc(tmem, kTmemCols);
+    if (warp == 8) tc_dealloc(tmem, kTmemCols);
 }
 
 bool attn_tc_supported(int H) { return H == 64 || H == 128; }

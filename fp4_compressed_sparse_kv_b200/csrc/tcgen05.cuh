@@ -30,6 +30,19 @@ __device__ __forceinline__ uint64_t umma_sdesc_sw128(uint32_t saddr, uint32_t lb
     return d;
 }
 
+// Shared-memory matrix descriptor without swizzle (canonical 8-row x 16-byte core matrices).  With
+// both strides 0 every core matrix reads the same 128 bytes, which makes a constant operand from one
+// 128-byte block.
+__device__ __forceinline__ uint64_t umma_sdesc_noswz(uint32_t saddr, uint32_t lbo, uint32_t sbo)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)((lbo & 0x3FFFFu) >> 4) << 16;
+    d |= (uint64_t)((sbo & 0x3FFFFu) >> 4) << 32;
+    d |= 1ull << 46;   // descriptor version; layout type 0 = no swizzle
+    return d;
+}
+
 __device__ __forceinline__ void tc_mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                            uint32_t accumulate)
 {
