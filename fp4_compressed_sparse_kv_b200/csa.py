@@ -56,7 +56,7 @@ class LayerStepC(ctypes.Structure):
 
 EXPORTS = ["csa_workspace_bytes", "csa_workspace_init", "csa_kv_pack_fp4", "csa_indexer_full",
            "csa_indexer_reindex", "csa_indexer_block_scores", "csa_topk_blocks", "csa_index_reuse", "csa_sparse_decode_attn", "csa_decode_layer",
-           "csa_check_device_error", "csa_status_string"]
+           "csa_check_device_error", "csa_status_string", "csa_indexer_full_noalloc"]
 
 _lib = None
 
@@ -97,6 +97,9 @@ def lib():
     L.csa_decode_layer.restype = st
     L.csa_decode_layer.argtypes = [ctypes.POINTER(KVLayerC), ctypes.POINTER(BatchC),
                                    ctypes.POINTER(LayerStepC), P, sz, P]
+    L.csa_indexer_full_noalloc.restype = st
+    L.csa_indexer_full_noalloc.argtypes = [ctypes.POINTER(KVLayerC), ctypes.POINTER(BatchC), P, P, i32, P, P,
+                                           P, P]
     L.csa_check_device_error.restype = st
     L.csa_check_device_error.argtypes = [P, P, ctypes.POINTER(ctypes.c_int64)]
     L.csa_status_string.restype = ctypes.c_char_p
@@ -274,6 +277,17 @@ def decode_layer(mode, layer, batch, q, out, lse, blocks, count, ws, iq=None, iw
                       _ptr(out, "out"), _ptr(lse, "lse"))
     _check(lib().csa_decode_layer(ctypes.byref(lc), ctypes.byref(bc), ctypes.byref(step),
                                   _ptr(ws, "ws"), ws.numel(), _stream(stream)), "csa_decode_layer")
+
+
+def indexer_full_noalloc(layer, batch, iq, iw, k, out_blocks, out_count, dev_status=None, stream=None):
+    """csa_indexer_full without a workspace: the library's own fixed scratch array is used instead, so
+    nothing is allocated.  For callers that cannot provide device memory; see include/csa.h for the
+    size limit and the rule that calls overlapping on the GPU must not share a device."""
+    lc, bc = layer.c(), batch.c()
+    _check(lib().csa_indexer_full_noalloc(ctypes.byref(lc), ctypes.byref(bc), _ptr(_bits(iq), "iq"),
+                                          _ptr(iw, "iw"), int(k), _ptr(out_blocks, "out_blocks"),
+                                          _ptr(out_count, "out_count"), _ptr(dev_status, "dev_status"),
+                                          _stream(stream)), "csa_indexer_full_noalloc")
 
 
 def check_device_error(ws, stream=None):

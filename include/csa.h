@@ -232,6 +232,29 @@ typedef struct {
 csa_status csa_decode_layer(const csa_kv_layer *layer, const csa_batch *batch,
                             const csa_layer_step *step, void *ws, size_t ws_bytes, void *stream);
 
+/*
+ * Full-layer indexer that allocates nothing (the pages have no counterpart to this entry point: it is
+ * an interface convenience).  Same inputs, outputs and results as csa_indexer_full, but the scratch it
+ * needs lives in a fixed array inside the library instead of a caller workspace, for callers that
+ * cannot obtain device memory where they run the indexer: runtimes with a fixed memory budget that
+ * forbid allocation after start-up, plugins inside a framework that owns the allocator, or paths that
+ * must not call an allocator at all.
+ *   dev_status  optional int32 device pointer (may be NULL): receives the device-data status code of
+ *               this call (0, or CSA_ERR_DEVICE_DATA / CSA_ERR_TIMEOUT), written asynchronously.
+ * Limit: 256 + 4 * B * max(ceil(max_seq_len / 8), k) bytes must fit in CSA_NOALLOC_SCRATCH_BYTES
+ * (4 MiB; e.g. 8 sequences of 131,072 tokens use 512 KiB); larger calls return CSA_ERR_WORKSPACE.
+ * Every GPU that loads the library holds that array until the process exits.  The first call on each
+ * device looks up the array's device address (cudaGetSymbolAddress, with that device current); make
+ * that first call before any stream capture.  All calls on a device share the one array and each call
+ * overwrites it: calls that overlap on the GPU (different streams without ordering between them) race
+ * and give undefined results.  No allocation or free happens in any call.
+ */
+#define CSA_NOALLOC_SCRATCH_BYTES (4 << 20)
+csa_status csa_indexer_full_noalloc(const csa_kv_layer *layer, const csa_batch *batch,
+                                    const uint16_t *iq, const float *iw, int32_t k,
+                                    int32_t *out_blocks, int32_t *out_count, int32_t *dev_status,
+                                    void *stream);
+
 /* Synchronise `stream`, read and clear the workspace status word.  Returns CSA_OK,
  * CSA_ERR_DEVICE_DATA or CSA_ERR_TIMEOUT; *detail (host, may be NULL) receives the first
  * offending index recorded. */
