@@ -40,6 +40,7 @@ def parse():
     ap.add_argument("--workload", default="decode_128k")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="time eager launches only")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU baseline sample budget")
     return ap.parse_args()
 
@@ -144,6 +145,25 @@ def traffic_from_profiles(call, workload):
     return None
 
 
+def max_over_ranks(value, device):
+    """The largest value over all ranks (the job's step time is its slowest rank's)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_workload(name, rank):
+    """Rank r's batch: the named workload's shape with its own seed (rank 0 keeps the base seed)."""
+    from fp4_compressed_sparse_kv_b200 import synth
+    w = synth.workload(name)
+    if rank > 0:
+        w.seed = (w.seed if isinstance(w.seed, list) else [w.seed]) + [rank]
+    return w
+
+
 def make_plan(st, scores_buf):
     """The step as a list of (call name, kernels launched, fn)."""
     from fp4_compressed_sparse_kv_b200 import csa
@@ -240,9 +260,7 @@ def run_ours(args, rank, world, local):
         dist.barrier()
     torch.cuda.set_device(local)
     dev = "cuda:%d" % local
-    w = synth.workload(args.workload)
-    if rank > 0:       # every rank processes its own batch of the same shape
-        w.seed = (w.seed if isinstance(w.seed, list) else [w.seed]) + [rank]
+    w = rank_workload(args.workload, rank)   # every rank processes its own batch of the same shape
     t0 = time.time()
     st = workloads.DecodeState(w, device=dev)
     setup_s = time.time() - t0
@@ -265,13 +283,36 @@ def run_ours(args, rank, world, local):
 
     K = args.steps
     names = [n for n, _, _ in plan]
+    # The step replayed as one CUDA graph (how a decode step runs in serving: no per-launch host
+    # overhead); fall back to eager launches if capture is not possible here.
+    graph = None
+    if not args.no_graph:
+        try:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                step()
+            for _ in range(args.warmup):
+                graph.replay()
+            torch.cuda.synchronize()
+            st.check()
+        except Exception as exc:  # noqa: BLE001 - report and continue eagerly
+            print("graph capture unavailable (%s); timing eager launches" % exc, file=sys.stderr)
+            graph = None
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(plan) + 1)] for _ in range(K)]
+    gev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     clocks = Clocks(local)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     clocks.start()
     wall0 = time.time()
+    if graph is not None:
+        for i in range(K):
+            flush.zero_()
+            gev[i][0].record(stream)
+            graph.replay()
+            gev[i][1].record(stream)
+    # per-call breakdown: the same step with eager launches and an event around every call
     for i in range(K):
         flush.zero_()
         for j, (_, _, fn) in enumerate(plan):
@@ -293,11 +334,9 @@ def run_ours(args, rank, world, local):
             per_call.setdefault(n, []).append(ev[i][j].elapsed_time(ev[i][j + 1]))
     call_ms = {n: sum(v) / K for n, v in per_call.items()}     # per step, summed over layers
     calls_per_step = {n: names.count(n) for n in set(names)}
-    mean_ms = sum(step_ms) / K
-    t = torch.tensor([mean_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
+    eager_ms = sum(step_ms) / K
+    mean_ms = sum(gev[i][0].elapsed_time(gev[i][1]) for i in range(K)) / K if graph is not None else eager_ms
+    max_ms = max_over_ranks(mean_ms, dev)
 
     # ---- end to end through the public API: pinned host inputs in, results out, every step
     B, H = w.batch, w.heads
@@ -337,10 +376,7 @@ def run_ours(args, rank, world, local):
         b_.record(stream)
         b_.synchronize()
         e_ms.append(a.elapsed_time(b_))
-    te = torch.tensor([sum(e_ms) / K], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te.item())
+    e2e_ms = max_over_ranks(sum(e_ms) / K, dev)
 
     if rank != 0:
         return None
@@ -378,7 +414,10 @@ def run_ours(args, rank, world, local):
         "kernels": kernels,
         "e2e": {"value": round(world * B / (e2e_ms * 1e-3), 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},
-        "gpu_launches": K * sum(k for _, k, _ in plan),
+        "gpu_launches": (2 if graph is not None else 1) * K * sum(k for _, k, _ in plan),
+        "timing": ("CUDA-graph replay of the step (headline); per-kernel figures from eager launches "
+                   "with an event around every call, eager step %.5f ms" % eager_ms) if graph is not None
+                  else "eager launches with an event around every call",
         "clocks": clk,
         "wall_s_timed": round(wall, 3),
         "setup_s": round(setup_s, 1),
