@@ -125,10 +125,11 @@ def source_sha(names):
     return h.hexdigest()[:12]
 
 
-KERNEL_SOURCES = {"indexer_block_scores": ["indexer.cu", "common.cuh", "convert.cuh", "pipeline.cuh"],
+KERNEL_SOURCES = {"indexer_full": ["screen.cu", "indexer.cu", "radix.cuh", "common.cuh", "convert.cuh", "pipeline.cuh",
+                                   "tcgen05.cuh"],
+                  "indexer_reindex": ["indexer.cu", "radix.cuh", "common.cuh", "convert.cuh", "pipeline.cuh"],
                   "sparse_decode_attn": ["attention_cc.cu", "attention_tc.cu", "attention_common.cuh", "tcgen05.cuh",
                                          "common.cuh", "convert.cuh"],
-                  "topk_blocks": ["indexer.cu", "common.cuh"],
                   "kv_pack_fp4": ["pack.cu", "common.cuh", "convert.cuh"]}
 
 
@@ -164,8 +165,8 @@ def rank_workload(name, rank):
     return w
 
 
-def make_plan(st, scores_buf):
-    """The step as a list of (call name, kernels launched, fn)."""
+def make_plan(st):
+    """The step as a list of (call name, kernels launched, fn): the library's public calls."""
     from fp4_compressed_sparse_kv_b200 import csa
     w = st.w
     plan = []
@@ -174,22 +175,17 @@ def make_plan(st, scores_buf):
         lay = st.layers[f]
         if m == csa.FULL:
             plan.append(("kv_pack_fp4", 1, lambda f=f: st.pack_new_tokens(f)))
-            plan.append(("indexer_block_scores", 1,
-                         lambda l=l, lay=lay: csa.indexer_block_scores(lay, st.batch, st.iq[l], st.iw[l],
-                                                                       scores_buf, st.ws)))
-            plan.append(("topk_blocks", 1,
-                         lambda l=l: csa.topk_blocks(st.batch, scores_buf, st.layer_k[l], st.blocks[l],
-                                                     st.count[l], st.ws)))
+            # qterm, screen, candidates, exact re-score, Top-K (one launch when every block is selected)
+            n_full = 1 if (st.max_seq_len + 7) // 8 <= st.layer_k[l] else 5
+            plan.append(("indexer_full", n_full,
+                         lambda l=l, lay=lay: csa.indexer_full(lay, st.batch, st.iq[l], st.iw[l], st.layer_k[l],
+                                                               st.blocks[l], st.count[l], st.ws)))
         elif m == csa.REINDEX:
             fl = st.full_of[l]
-            plan.append(("indexer_block_scores", 1,
-                         lambda l=l, lay=lay, fl=fl: csa.indexer_block_scores(
-                             lay, st.batch, st.iq[l], st.iw[l], scores_buf, st.ws, pool=st.blocks[fl],
-                             pool_count=st.count[fl])))
-            plan.append(("topk_blocks", 1,
-                         lambda l=l, fl=fl: csa.topk_blocks(st.batch, scores_buf, st.layer_k[l], st.blocks[l],
-                                                            st.count[l], st.ws, pool=st.blocks[fl],
-                                                            pool_count=st.count[fl])))
+            plan.append(("indexer_reindex", 2,
+                         lambda l=l, lay=lay, fl=fl: csa.indexer_reindex(
+                             lay, st.batch, st.iq[l], st.iw[l], st.blocks[fl], st.count[fl], st.layer_k[l],
+                             st.blocks[l], st.count[l], st.ws)))
         else:
             plan.append(("index_reuse", 1,
                          lambda l=l: csa.index_reuse(st.blocks[l - 1], st.count[l - 1], st.blocks[l],
@@ -216,12 +212,12 @@ def algorithmic_bytes(st):
     for l, m in enumerate(w.modes):
         if m == 0:
             add("kv_pack_fp4", B * (1024 + 256 + 256 + 32 + 128 + 512 + 4 + 12))
-            add("indexer_block_scores", (lens * 128).sum() + ((lens + 7) // 8).sum() * 4 + B * (2048 + 32))
-            add("topk_blocks", ((lens + 7) // 8).sum() * 4 + B * st.layer_k[l] * 4)
+            # every key once, the queries and weights, the selected ids
+            add("indexer_full", (lens * 128).sum() + B * (2048 + 32) + B * st.layer_k[l] * 4)
         elif m == 1:
             pc = st.count[st.full_of[l]].cpu().numpy().astype(np.int64)
-            add("indexer_block_scores", (pc * 8 * 128).sum() + pc.sum() * 8 + B * (2048 + 32))
-            add("topk_blocks", pc.sum() * 8 + B * st.layer_k[l] * 4)
+            # the pool's keys, the pool ids, the queries and weights, the selected ids
+            add("indexer_reindex", (pc * 8 * 128).sum() + pc.sum() * 4 + B * (2048 + 32) + B * st.layer_k[l] * 4)
         else:
             add("index_reuse", st.count[l - 1].cpu().numpy().sum() * 8)
         blocks = st.blocks[l].cpu().numpy()
@@ -264,9 +260,7 @@ def run_ours(args, rank, world, local):
     t0 = time.time()
     st = workloads.DecodeState(w, device=dev)
     setup_s = time.time() - t0
-    nb_max = (st.max_seq_len + 7) // 8
-    scores_buf = torch.zeros((w.batch, max(nb_max, st.cap)), dtype=torch.float32, device=dev)
-    plan = make_plan(st, scores_buf)
+    plan = make_plan(st)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
@@ -391,11 +385,21 @@ def run_ours(args, rank, world, local):
                       "hbm_frac": round(gbs / peaks["hbm_gbs"], 4)}
     per_launch_ms = call_ms[dominant] / calls_per_step[dominant]
     per_launch_bytes = bytes_per_call[dominant] / calls_per_step[dominant]
-    achieved = per_launch_bytes / (per_launch_ms * 1e-3) / 1e9
+    per_launch_flops = (flops_attn if dominant == "sparse_decode_attn" else 0.0) / calls_per_step[dominant]
     traffic = traffic_from_profiles(dominant, args.workload)
-    roof = {"bound": "hbm", "kernel": dominant, "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
-            "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-            "traffic": traffic, "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs)"}
+    # the bound is whichever floor is higher: bytes at the measured copy bandwidth or FLOPs at the
+    # measured dense tensor rate (f16 operands run at the bf16 rate)
+    if per_launch_flops / (peaks["bf16_tflops"] * 1e12) > per_launch_bytes / (peaks["hbm_gbs"] * 1e9):
+        achieved = per_launch_flops / (per_launch_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "kernel": dominant, "achieved": round(achieved, 1), "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": traffic,
+                "peak_source": peaks["source"] + " (MEASURED_PEAKS.json bf16_tflops, burst; f16 same rate)",
+                "bytes_frac": round(per_launch_bytes / (per_launch_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
+    else:
+        achieved = per_launch_bytes / (per_launch_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "kernel": dominant, "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": traffic, "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs)"}
     step_bytes = sum(bytes_per_call.values())
     attn_ms = call_ms.get("sparse_decode_attn", 0.0)
     line = {

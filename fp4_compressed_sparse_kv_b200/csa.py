@@ -56,7 +56,8 @@ class LayerStepC(ctypes.Structure):
 
 EXPORTS = ["csa_workspace_bytes", "csa_workspace_init", "csa_kv_pack_fp4", "csa_indexer_full",
            "csa_indexer_reindex", "csa_indexer_block_scores", "csa_topk_blocks", "csa_index_reuse", "csa_sparse_decode_attn", "csa_decode_layer",
-           "csa_check_device_error", "csa_status_string", "csa_indexer_full_noalloc"]
+           "csa_check_device_error", "csa_status_string", "csa_indexer_full_noalloc",
+           "csa_indexer_screen_bounds"]
 
 _lib = None
 
@@ -87,6 +88,9 @@ def lib():
     L.csa_indexer_block_scores.restype = st
     L.csa_indexer_block_scores.argtypes = [ctypes.POINTER(KVLayerC), ctypes.POINTER(BatchC), P, P, P, P,
                                            i32, P, i32, P, sz, P]
+    L.csa_indexer_screen_bounds.restype = st
+    L.csa_indexer_screen_bounds.argtypes = [ctypes.POINTER(KVLayerC), ctypes.POINTER(BatchC), P, P, P, P,
+                                            i32, P, sz, P]
     L.csa_topk_blocks.restype = st
     L.csa_topk_blocks.argtypes = [ctypes.POINTER(BatchC), P, i32, P, P, i32, i32, P, P, P, sz, P]
     L.csa_index_reuse.restype = st
@@ -233,6 +237,18 @@ def indexer_block_scores(layer, batch, iq, iw, scores, ws, pool=None, pool_count
                                           int(pool.shape[1]) if pool is not None else 0,
                                           _ptr(scores, "scores"), int(scores.shape[1]), _ptr(ws, "ws"),
                                           ws.numel(), _stream(stream)), "csa_indexer_block_scores")
+
+
+def indexer_screen_bounds(layer, batch, iq, iw, lower, upper, ws, stream=None):
+    """Per-block bounds of the exact Full score from the tensor-core screen: float32 [B, stride] each,
+    lower <= score <= upper in Top-K order (-NaN / +NaN where no bound could be formed)."""
+    lc, bc = layer.c(), batch.c()
+    if lower.shape != upper.shape:
+        raise ValueError("lower and upper must have the same shape")
+    _check(lib().csa_indexer_screen_bounds(ctypes.byref(lc), ctypes.byref(bc), _ptr(_bits(iq), "iq"),
+                                           _ptr(iw, "iw"), _ptr(lower, "lower"), _ptr(upper, "upper"),
+                                           int(lower.shape[1]), _ptr(ws, "ws"), ws.numel(), _stream(stream)),
+           "csa_indexer_screen_bounds")
 
 
 def topk_blocks(batch, scores, k, out_blocks, out_count, ws, pool=None, pool_count=None, stream=None):

@@ -19,6 +19,20 @@ cudaError_t launch_block_scores_full_or_pool(const uint8_t *keys, int num_pages,
                                              const uint16_t *iq, const float *iw, const int32_t *pool,
                                              const int32_t *pool_count, int pool_cap, float *scores,
                                              int score_stride, void *ws, cudaStream_t st);
+cudaError_t launch_block_scores_list(const uint8_t *keys, int num_pages, const csa_batch &bt, const uint16_t *iq,
+                                     const float *iw, const uint2 *list, const int32_t *list_count, float *scores,
+                                     int score_stride, void *ws, cudaStream_t st);
+bool screen_supported(int num_pages);
+cudaError_t launch_screen_bounds(const uint8_t *keys, int num_pages, const csa_batch &bt, const uint16_t *iq,
+                                 const float *iw, uint8_t *qt, void *qm, int32_t *list_count, uint32_t *hist,
+                                 uint32_t *hist2, void *words, float *lo, float *hi, int stride, void *ws,
+                                 cudaStream_t st);
+cudaError_t launch_classify(const float *lo, const float *hi, int stride, const csa_batch &bt, int k,
+                            const uint32_t *hist, uint32_t *hist2, void *words, uint8_t *status, int sstride,
+                            int32_t *uslice, uint2 *list, int32_t *list_count, void *ws, cudaStream_t st);
+cudaError_t launch_finalize(const float *scores, int score_stride, const csa_batch &bt, uint8_t *status,
+                            int sstride, const int32_t *uslice, const void *words, int stride, int k,
+                            int32_t *out_blocks, int32_t *out_count, void *ws, cudaStream_t st);
 cudaError_t launch_attn_tc(const AttnArgs &a, cudaStream_t st);
 bool attn_tc_supported(int H);
 int attn_units_per_tile(int H);
@@ -155,13 +169,66 @@ csa_status csa_indexer_full(const csa_kv_layer *layer, const csa_batch *batch, c
     if (s != CSA_OK) return s;
     if (k < 1 || k > CSA_MAX_TOPK) return CSA_ERR_INVALID_ARG;
     const WsLayout w = ws_layout(batch->B, 16, batch->max_seq_len, k, 1);
-    if (ws_bytes < w.topk) return CSA_ERR_WORKSPACE;
-    float *scores = reinterpret_cast<float *>((char *)ws + w.scores);
-    s = csa_indexer_block_scores(layer, batch, iq, iw, nullptr, nullptr, 0, scores, (int32_t)w.score_cap, ws,
-                                 ws_bytes, stream);
-    if (s != CSA_OK) return s;
-    return csa_topk_blocks(batch, scores, (int32_t)w.score_cap, nullptr, nullptr, 0, k, out_blocks, out_count, ws,
-                           ws_bytes, stream);
+    if (ws_bytes < w.screen_end) return CSA_ERR_WORKSPACE;
+    cudaStream_t st = (cudaStream_t)stream;
+    char *base = (char *)ws;
+    float *scores = reinterpret_cast<float *>(base + w.scores);
+    const int nb = (int)w.nb;
+    if (nb <= k) {   // every sequence selects all of its blocks: no score is needed
+        return cuda_status(launch_topk(scores, (int)w.score_cap, batch->seq_len, batch->max_seq_len, nullptr, nullptr,
+                                       0, k, batch->B, out_blocks, out_count, nb, ws, st));
+    }
+    if (!screen_supported(layer->num_pages)) {   // exhaustive exact scan
+        s = csa_indexer_block_scores(layer, batch, iq, iw, nullptr, nullptr, 0, scores, (int32_t)w.score_cap, ws,
+                                     ws_bytes, stream);
+        if (s != CSA_OK) return s;
+        return csa_topk_blocks(batch, scores, (int32_t)w.score_cap, nullptr, nullptr, 0, k, out_blocks, out_count,
+                               ws, ws_bytes, stream);
+    }
+    // screen every position on the tensor cores; blocks sure to be in the Top-k are kept, blocks that
+    // cannot reach it dropped, the uncertain rest scored exactly and the best of them taken
+    float *lo = reinterpret_cast<float *>(base + w.lo);
+    float *hi = reinterpret_cast<float *>(base + w.hi);
+    uint32_t *hist = reinterpret_cast<uint32_t *>(base + w.hist);
+    uint32_t *hist2 = reinterpret_cast<uint32_t *>(base + w.hist2);
+    void *words = base + w.topk;
+    uint8_t *status = reinterpret_cast<uint8_t *>(base + w.status);
+    int32_t *uslice = reinterpret_cast<int32_t *>(base + w.uslice);
+    uint2 *list = reinterpret_cast<uint2 *>(base + w.list);
+    int32_t *list_count = reinterpret_cast<int32_t *>(base + w.list_count);
+    cudaError_t e = launch_screen_bounds(layer->keys, layer->num_pages, *batch, iq, iw,
+                                         reinterpret_cast<uint8_t *>(base + w.qt), base + w.qm, list_count, hist,
+                                         hist2, words, lo, hi, nb, ws, st);
+    if (e == cudaSuccess)
+        e = launch_classify(lo, hi, nb, *batch, k, hist, hist2, words, status, (int)w.status_stride, uslice, list,
+                            list_count, ws, st);
+    if (e == cudaSuccess)
+        e = launch_block_scores_list(layer->keys, layer->num_pages, *batch, iq, iw, list, list_count, scores,
+                                     (int)w.score_cap, ws, st);
+    if (e == cudaSuccess)
+        e = launch_finalize(scores, (int)w.score_cap, *batch, status, (int)w.status_stride, uslice, words, nb, k,
+                            out_blocks, out_count, ws, st);
+    return cuda_status(e);
+}
+
+csa_status csa_indexer_screen_bounds(const csa_kv_layer *layer, const csa_batch *batch, const uint16_t *iq,
+                                     const float *iw, float *lower, float *upper, int32_t stride, void *ws,
+                                     size_t ws_bytes, void *stream)
+{
+    if (!layer_ok(layer, false) || !batch_ok(batch)) return CSA_ERR_INVALID_ARG;
+    if (!iq || !iw || !lower || !upper || !ws || !aligned16(iq) || !aligned16(iw) || !aligned16(lower) ||
+        !aligned16(upper) || !aligned16(ws))
+        return CSA_ERR_INVALID_ARG;
+    const WsLayout w = ws_layout(batch->B, 16, batch->max_seq_len, 1, 1);
+    if (stride < (int32_t)w.nb) return CSA_ERR_INVALID_ARG;
+    if (!screen_supported(layer->num_pages)) return CSA_ERR_UNSUPPORTED;
+    if (ws_bytes < w.screen_end) return CSA_ERR_WORKSPACE;
+    char *base = (char *)ws;
+    return cuda_status(launch_screen_bounds(layer->keys, layer->num_pages, *batch, iq, iw,
+                                            reinterpret_cast<uint8_t *>(base + w.qt), base + w.qm,
+                                            reinterpret_cast<int32_t *>(base + w.list_count),
+                                            reinterpret_cast<uint32_t *>(base + w.hist), nullptr, nullptr, lower, upper,
+                                            stride, ws, (cudaStream_t)stream));
 }
 
 csa_status csa_indexer_reindex(const csa_kv_layer *layer, const csa_batch *batch, const uint16_t *iq,

@@ -20,7 +20,9 @@ constexpr int kIdxDim = CSA_INDEX_DIM;
 constexpr int kWindow = CSA_WINDOW;
 
 // ------------------------------------------------------------------------------------------------
-// Workspace: [0, 256) status header; then block scores; then attention split partials.
+// Workspace: [0, 256) status header; then block scores; the Full indexer's screening buffers; then
+// attention split partials.  Offsets up to the attention partials depend on B, max_seq_len and cap
+// only, so indexer calls need not know H.
 // ------------------------------------------------------------------------------------------------
 constexpr size_t kHeaderBytes = CSA_WORKSPACE_HEADER_BYTES;
 constexpr int kNumSms = 148;                // B200 SM count, used to size the attention split
@@ -31,6 +33,18 @@ struct WsLayout {
     size_t scores = 0;       // float [B][score_cap]
     size_t score_cap = 0;
     size_t topk = 0;         // uint32 [B][topk_words] per-sequence select state
+    size_t nb = 0;           // blocks of the longest sequence
+    size_t lo = 0, hi = 0;   // float [B][nb] screening bounds of every block
+    size_t qt = 0;           // uint8 [B][kQtBytes] query-term operand images
+    size_t qm = 0;           // [B][kQmBytes] per-sequence screening constants
+    size_t status = 0;       // uint8 [B][status_stride] class of every block (out, sure, uncertain, ...)
+    size_t status_stride = 0;   // nb rounded up to 16
+    size_t uslice = 0;       // int32 [B][nb] each sequence's uncertain blocks, any order
+    size_t list = 0;         // uint2 [B * nb] re-scoring work list (b, block)
+    size_t list_count = 0;   // int32 entries in the list
+    size_t hist = 0;         // uint32 [B][kHistBins] histogram of the blocks' lower-bound keys
+    size_t hist2 = 0;        // uint32 [B][kHistBins] second level, inside the threshold bin
+    size_t screen_end = 0;   // end of the indexer's regions
     size_t part_o = 0;       // float [B][splits][H][512]
     size_t part_ml = 0;      // float2 [B][splits][H]  (running max, running sum)
     int splits = 0;
@@ -55,6 +69,9 @@ inline int attn_splits(int B, int cap, int units_per_tile)
 }
 
 constexpr int kTopkWords = 4;
+constexpr size_t kQtBytes = 32 * CSA_INDEX_DIM;   // 3 E4M3 terms x 8 heads + 8 zero rows, 128 B each
+constexpr size_t kQmBytes = 64;
+constexpr int kHistBins = 4096;                   // top 12 bits of a 32-bit order key
 
 inline WsLayout ws_layout(int B, int H, int max_seq_len, int cap, int units_per_tile)
 {
@@ -66,6 +83,29 @@ inline WsLayout ws_layout(int B, int H, int max_seq_len, int cap, int units_per_
     o = align_up(o + (size_t)B * w.score_cap * 4, 256);
     w.topk = o;
     o = align_up(o + (size_t)B * kTopkWords * 4, 256);
+    w.nb = nb;
+    w.lo = o;
+    o = align_up(o + (size_t)B * nb * 4, 256);
+    w.hi = o;
+    o = align_up(o + (size_t)B * nb * 4, 256);
+    w.qt = o;
+    o = align_up(o + (size_t)B * kQtBytes, 1024);
+    w.qm = o;
+    o = align_up(o + (size_t)B * kQmBytes, 256);
+    w.status = o;
+    w.status_stride = align_up(nb, 16);
+    o = align_up(o + (size_t)B * w.status_stride, 256);
+    w.uslice = o;
+    o = align_up(o + (size_t)B * nb * 4, 256);
+    w.list = o;
+    o = align_up(o + (size_t)B * nb * 8, 256);
+    w.list_count = o;
+    o = align_up(o + 4, 256);
+    w.hist = o;
+    o = align_up(o + (size_t)B * kHistBins * 4, 256);
+    w.hist2 = o;
+    o = align_up(o + (size_t)B * kHistBins * 4, 256);
+    w.screen_end = o;
     w.splits = attn_splits(B, cap, units_per_tile);
     w.part_o = o;
     o = align_up(o + (size_t)B * w.splits * H * kLatent * 4, 256);

@@ -10,13 +10,16 @@
 #include "common.cuh"
 #include "convert.cuh"
 #include "pipeline.cuh"
+#include "radix.cuh"
 
 namespace csa {
 
 // ------------------------------------------------------------------------------------------------
 // Block scoring.  Persistent CTAs of 8 warps; a work item is 8 consecutive "virtual" blocks of one
 // sequence (in Full mode virtual block v is block v, so an item is one 64-token page; in Reindex
-// mode it is pool[b][v]) and warp w always takes virtual block w of each item.  Every warp runs its
+// mode it is pool[b][v]) and warp w always takes virtual block w of each item.  In list mode an item
+// is 8 consecutive entries (b, block) of a device-built work list, warp w taking entry w, and the
+// score goes to scores[b][block]; the list holds only real work.  Every warp runs its
 // own pipeline: lane 0 resolves the block's page a few items ahead and bulk-copies its 1 KB of keys
 // into the warp's shared-memory ring; no warp ever waits for another.
 //
@@ -47,6 +50,8 @@ struct ScoreArgs {
     const int32_t *pool_count;
     int pool_cap;
     int items_per_seq;
+    const uint2 *list;          // list mode: entries (b, block), count in *list_count
+    const int32_t *list_count;
     float *scores;
     int score_stride;
     void *ws;
@@ -133,7 +138,13 @@ __global__ void __launch_bounds__(kScoreThreads, 1) block_score_kernel(ScoreArgs
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     ScoreSmem &sm = *reinterpret_cast<ScoreSmem *>(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long total = (long long)a.B * a.items_per_seq;
+    const long long total =
+        a.list ? ((long long)max(*a.list_count, 0) + kScoreWarps - 1) / kScoreWarps : (long long)a.B * a.items_per_seq;
+    // each CTA takes a contiguous range of items, so consecutive items mostly share a sequence (and
+    // its query stays in registers)
+    const long long per = (total + gridDim.x - 1) / gridDim.x;
+    const long long first = (long long)blockIdx.x * per;
+    const long long last = first + per < total ? first + per : total;
 
     if (threadIdx.x == 0) {
         for (int w = 0; w < kScoreWarps; ++w)
@@ -146,9 +157,35 @@ __global__ void __launch_bounds__(kScoreThreads, 1) block_score_kernel(ScoreArgs
     // ---- metadata of this warp's block of items k0 .. k0+31, one item per lane, loads in parallel
     auto resolve32 = [&](long long k0) {
         const long long k = k0 + lane;
-        const long long item = blockIdx.x + k * (long long)gridDim.x;
+        const long long item = first + k;
         ItemMeta m{nullptr, 0, 0, kBlkEmpty, 0};
-        if (item < total) {
+        if (a.list) {
+            const long long e = item * kScoreWarps + warp;
+            if (item < last && e < *a.list_count) {
+                const uint2 ent = a.list[e];
+                const int b = (int)ent.x;
+                int blk = (int)ent.y;
+                const int L = (b >= 0 && b < a.B) ? a.seq_len[b] : 0;
+                const int nb = (L + kBlock - 1) / kBlock;
+                if (b < 0 || b >= a.B || blk < 0 || blk >= a.score_stride) {
+                    report(a.ws, CSA_ERR_DEVICE_DATA, e);
+                    sm.meta[warp][k % kMetaRing] = m;
+                    return;
+                }
+                m.b = b;
+                m.L = L;
+                m.v = blk;
+                const bool ok = L >= 1 && L <= a.max_seq_len && blk >= 0 && blk < nb;
+                const int page = ok ? a.block_table[(size_t)b * a.max_pages + blk / kBlocksPerPage] : -1;
+                if (page < 0 || page >= a.num_pages) {
+                    report(a.ws, CSA_ERR_DEVICE_DATA, e);
+                    blk = kBlkBad;
+                } else {
+                    m.src = a.keys + ((size_t)page * kPage + (size_t)(blk % kBlocksPerPage) * kBlock) * kIdxDim;
+                }
+                m.blk = blk;
+            }
+        } else if (item < last) {
             const int b = (int)(item / a.items_per_seq);
             const int grp = (int)(item % a.items_per_seq);
             const int L = a.seq_len[b];
@@ -190,8 +227,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1) block_score_kernel(ScoreArgs
     };
     // lane 0: start the copy of item k's block into stage k % kScoreStages
     auto issue = [&](long long k) {
-        const long long item = blockIdx.x + k * (long long)gridDim.x;
-        if (item >= total) return;
+        const long long item = first + k;
+        if (item >= last) return;
         const int st = (int)(k % kScoreStages);
         const ItemMeta &m = sm.meta[warp][k % kMetaRing];
         if (m.src) {
@@ -214,7 +251,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) block_score_kernel(ScoreArgs
     int cur_b = -1;
     const int g = lane >> 3, j = lane & 7;
     long long k = 0;
-    for (long long item = blockIdx.x; item < total; item += gridDim.x, ++k) {
+    for (long long item = first; item < last; ++item, ++k) {
         const long long kn = k + kScoreStages - 1;   // the item whose copy starts now
         if ((kn & 31) == 0) {
             resolve32(kn);
@@ -252,7 +289,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) block_score_kernel(ScoreArgs
             const float s0 = score_key(q2, w, kr0, lane);
             const float s1 = score_key(q2, w, kr1, lane);
             float best = -INFINITY;
-            if (m.blk * kBlock + g < m.L) best = s0;
+            if (m.blk * kBlock + g < m.L) best = fmaxf(best, s0);   // a NaN score never wins
             if (m.blk * kBlock + 4 + g < m.L) best = fmaxf(best, s1);
             best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, 8));
             best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, 16));
@@ -266,8 +303,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1) block_score_kernel(ScoreArgs
     // warp started (k counts the items consumed; issue() ran up to k + kScoreStages - 2)
     if (lane == 0) {
         for (long long kk = k; kk < k + kScoreStages - 1; ++kk) {
-            const long long item = blockIdx.x + kk * (long long)gridDim.x;
-            if (item >= total) break;
+            const long long item = first + kk;
+            if (item >= last) break;
             volatile int no_abort = 0;
             mbar_wait(&sm.full[warp][kk % kScoreStages], (uint32_t)((kk / kScoreStages) & 1), &no_abort, a.ws, -1);
         }
@@ -287,31 +324,6 @@ constexpr int kTopkThreads = 1024;
 constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kTopkCacheKeys = 16384;
 constexpr int kTopkHistWords = kTopkWarps * 256;
-
-__device__ __forceinline__ uint32_t block_reduce_minmax(uint32_t v, bool is_max, uint32_t *scratch)
-{
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        const uint32_t y = __shfl_xor_sync(0xffffffffu, v, o);
-        v = is_max ? max(v, y) : min(v, y);
-    }
-    if (lane == 0) scratch[warp] = v;
-    __syncthreads();
-    if (warp == 0) {
-        v = scratch[lane];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const uint32_t y = __shfl_xor_sync(0xffffffffu, v, o);
-            v = is_max ? max(v, y) : min(v, y);
-        }
-        if (lane == 0) scratch[32] = v;
-    }
-    __syncthreads();
-    v = scratch[32];
-    __syncthreads();
-    return v;
-}
 
 __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const float *__restrict__ scores, int score_stride,
                                                                const int32_t *__restrict__ seq_len, int max_seq_len,
@@ -348,66 +360,13 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const float *__re
         return;
     }
     const bool cached = n <= kTopkCacheKeys;
-    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-    for (int i = t; i < n; i += kTopkThreads) {
-        const uint32_t u = order_key(sc[i]);
-        if (cached) skeys[i] = u;
-        kmin = min(kmin, u);
-        kmax = max(kmax, u);
+    if (cached) {
+        for (int i = t; i < n; i += kTopkThreads) skeys[i] = order_key(sc[i]);
+        __syncthreads();
     }
-    kmin = block_reduce_minmax(kmin, false, scratch);
-    kmax = block_reduce_minmax(kmax, true, scratch);
-
-    uint32_t prefix = kmax, mask = 0xFFFFFFFFu, remaining = (uint32_t)k;
-    if (kmin != kmax) {
-        int hi = 31 - __clz(kmin ^ kmax);              // highest bit that differs between keys
-        mask = hi == 31 ? 0u : ~((2u << hi) - 1u);
-        prefix = kmax & mask;
-        while (hi >= 0) {
-            const int width = hi + 1 < 8 ? hi + 1 : 8;
-            const int shift = hi + 1 - width;
-            const uint32_t dmask = (1u << width) - 1u;
-            for (int i = t; i < kTopkHistWords; i += kTopkThreads) whist[i] = 0u;
-            __syncthreads();
-            for (int i = t; i < n; i += kTopkThreads) {
-                const uint32_t u = cached ? skeys[i] : order_key(sc[i]);
-                if ((u & mask) == prefix) atomicAdd(&whist[warp * 256 + ((u >> shift) & dmask)], 1u);
-            }
-            __syncthreads();
-            // bin totals, then counts from the top bin down; the threshold bin is where they reach
-            // `remaining`
-            uint32_t c = 0;
-            if (t < 256) {
-                const int bin = 255 - t;
-#pragma unroll 8
-                for (int w = 0; w < kTopkWarps; ++w) c += whist[w * 256 + bin];
-            }
-            uint32_t x = c;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-                if (lane >= o) x += y;
-            }
-            if (t < 256 && lane == 31) scratch[warp] = x;
-            __syncthreads();
-            if (t < 256) {
-                uint32_t before = 0;
-                for (int wi = 0; wi < warp; ++wi) before += scratch[wi];
-                const uint32_t incl = before + x;
-                if (incl >= remaining && incl - c < remaining) {
-                    sel[0] = 255u - (uint32_t)t;
-                    sel[1] = incl - c;
-                }
-            }
-            __syncthreads();
-            prefix |= sel[0] << shift;
-            mask |= dmask << shift;
-            remaining -= sel[1];
-            hi = shift - 1;
-            __syncthreads();
-        }
-    }
-    const uint32_t T = prefix, need_eq = remaining;
+    uint32_t T, need_eq;
+    radix_select<kTopkThreads>(n, (uint32_t)k, [&](int i) { return cached ? skeys[i] : order_key(sc[i]); }, 0, whist,
+                               scratch, sel, T, need_eq);
 
     // per-warp contiguous segments: counts, then ordered writes
     const int seg = (n + kTopkWarps - 1) / kTopkWarps;
@@ -511,10 +470,45 @@ cudaError_t launch_block_scores_full_or_pool(const uint8_t *keys, int num_pages,
     a.pool_cap = pool_cap;
     a.items_per_seq = pool ? (pool_cap + kScoreWarps - 1) / kScoreWarps
                            : (bt.max_seq_len + kPage - 1) / kPage;
+    a.list = nullptr;
+    a.list_count = nullptr;
     a.scores = scores;
     a.score_stride = score_stride;
     a.ws = ws;
     return launch_block_scores(a, st);
+}
+
+// Exact scores of the blocks named by a device-built work list: entry (b, blk) scores block blk of
+// sequence b into scores[b][blk].  The list and count come from this library's own kernels (seq_len,
+// block table and pages are still checked).
+cudaError_t launch_block_scores_list(const uint8_t *keys, int num_pages, const csa_batch &bt, const uint16_t *iq,
+                                     const float *iw, const uint2 *list, const int32_t *list_count, float *scores,
+                                     int score_stride, void *ws, cudaStream_t st)
+{
+    ScoreArgs a;
+    a.keys = keys;
+    a.num_pages = num_pages;
+    a.seq_len = bt.seq_len;
+    a.block_table = bt.block_table;
+    a.max_pages = bt.max_pages;
+    a.max_seq_len = bt.max_seq_len;
+    a.B = bt.B;
+    a.iq = iq;
+    a.iw = iw;
+    a.pool = nullptr;
+    a.pool_count = nullptr;
+    a.pool_cap = 0;
+    a.items_per_seq = 0;
+    a.list = list;
+    a.list_count = list_count;
+    a.scores = scores;
+    a.score_stride = score_stride;
+    a.ws = ws;
+    const size_t smem = sizeof(ScoreSmem);
+    cudaError_t e = cudaFuncSetAttribute(block_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    block_score_kernel<<<num_sms(), kScoreThreads, smem, st>>>(a);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_topk(const float *scores, int score_stride, const int32_t *seq_len, int max_seq_len,

@@ -1,0 +1,986 @@
+// screen.cu -- the Full-layer indexer's tensor-core screening: per-block bounds of the exact score,
+// and from them the candidate blocks that must be scored exactly.
+//
+// rebasdaily article on DeepSeek-V4.1-Flash KV compression, section "同一份笔记，多层一起用": a Full
+// layer selects its Top-K blocks of 8 positions over the whole context, so its scan reads every
+// indexer key.  The exact score (csa.h) is a fixed binary32 FMA chain on CUDA cores; here every
+// position is first scored approximately on the tensor cores, at the speed of reading the keys, with
+// a rigorous bound eps on the distance to the exact score.  The exact Top-K lies among the blocks
+// whose upper bound reaches the k-th largest lower bound; only those are scored exactly
+// (csa_indexer_full), so the result is identical to the exhaustive exact scan.
+//
+//  1. qterm_kernel: per sequence and head, q_h * 2^s (largest |q| in [128, 256)) is split into three
+//     E4M3 terms t1 + t2 + t3 plus a residual delta, and written as the tensor-core B operand.
+//  2. screen_kernel: D_i = t_i . k for all positions from tcgen05 MMAs (kind::f8f6f4, E4M3 x E4M3,
+//     fp32 accumulation in TMEM) on key tiles brought in by TMA; the epilogue forms the approximate
+//     head values d^_h = ((D_1 + D_2) + D_3) 2^-s, the approximate score t^ = the same weighted ReLU
+//     chain as the exact score, the bound eps_p, then per block the largest lower and upper bound,
+//     and a per-sequence histogram of the lower bounds.
+//  3. classify_a/b_kernel: thresholds T and U from the histograms and the widest interval, then each
+//     block is out, sure (certainly in the Top-K) or uncertain; uncertain blocks go to a work list.
+//  4. (indexer.cu) the exact scorer scores the uncertain blocks.
+//  5. finalize_kernel: the sure blocks plus the best uncertain ones, in ascending block order.
+
+// The bound, with u = 2^-24, gamma_n = n u / (1 - n u), kmax_p the position's largest |key|:
+//  * exact chain: 16-term FMA chains then a 3-level tree; every product bf16 x E4M3 is exact in
+//    binary32, so |d_h - q_h . k| <= gamma_19 sum_d |q_d k_d| <= gamma_19 kmax Q1_h (Q1_h = sum |q_d|);
+//  * screen: the tensor core's fp32 accumulation is taken to err by at most kTcRel times the sum of
+//    the magnitudes of its (exact) products -- measured on B200 below 2^-25 for E4M3, taken as 2^-14;
+//    then two binary32 adds and an exact power-of-two scale:
+//    |d^_h - q_h . k| <= kmax ((kTcRel + gamma_2 (1 + kTcRel)) T1_h + Delta_h), with T1_h the sum of
+//    all |t_i,d| 2^-s and Delta_h = sum |delta_d| 2^-s;
+//  * so |d^_h - d_h| <= kmax F_h, F_h = (kTcRel + gamma_2 (1 + kTcRel)) T1_h + Delta_h + gamma_19 Q1_h;
+//    ReLU is 1-Lipschitz and both weighted chains carry gamma_8 relative error, which gives
+//    |score - t^| <= kmax (1 + gamma_8) sum_h |w_h| F_h + 2 gamma_8 (1 + gamma_8) sum_h |w_h| relu(d^_h);
+//  * underflow adds at most a few 2^-150 per operation: an absolute slack 2^-100 (1 + sum |w|) covers
+//    it; positions where any partial sum could come near overflow (kmax Q1 sum|w| >= 1e37) and
+//    non-finite values get no bound (lower = -NaN, upper = +NaN: the two ends of the Top-K order).
+// All constants are formed in double and rounded up by a relative 1e-6; the per-position sums use
+// round-up arithmetic.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "convert.cuh"
+#include "pipeline.cuh"
+#include "radix.cuh"
+#include "tcgen05.cuh"
+
+namespace csa {
+
+constexpr int kScrRows = 128;                             // positions per tile: two pages
+constexpr int kScrN = 32;                                 // MMA N: 3 terms x 8 heads + 8 zero rows
+constexpr int kScrStages = 9;
+constexpr int kScrEpiGroups = 2;                          // epilogue groups, taking tiles in turn
+constexpr int kScrAcc = 6;                                // TMEM accumulators (a multiple of the groups)
+constexpr int kScrTmemCols = 256;                         // >= 32 * kScrAcc, a power of two
+constexpr int kScrMaxGroups = 2;                          // row-max groups, taking tiles in turn
+constexpr int kScrThreads = 64 + 128 * kScrMaxGroups + 128 * kScrEpiGroups;   // loader, MMA, row max, epilogues
+constexpr int kScrEpiWarp0 = 2 + 4 * kScrMaxGroups;        // first epilogue warp
+static_assert(kScrAcc % kScrEpiGroups == 0, "each accumulator belongs to one epilogue group");
+static_assert(32 * kScrAcc <= kScrTmemCols, "accumulators must fit the TMEM allocation");
+constexpr uint32_t kScrKeyBytes = kScrRows * kIdxDim;     // 16 KB
+constexpr uint32_t kScrPageBytes = kPage * kIdxDim;       // 8 KB
+constexpr uint32_t kScrQtBytes = (uint32_t)kQtBytes;      // 4 KB
+constexpr int kScrRing = 64;                              // resolved-item ring (>= 32 + stages)
+constexpr double kTcRel = 6.103515625e-05;                // 2^-14
+constexpr double kU = 5.9604644775390625e-08;             // 2^-24
+constexpr double kRoundUp = 1.000001;
+
+__host__ __device__ constexpr double gamma_n(int n) { return n * kU / (1.0 - n * kU); }
+
+struct QMeta {
+    float inv_scale[8];   // 2^-s_h
+    float G;              // (1 + gamma_8) sum_h |w_h| F_h, rounded up
+    float chain;          // 2 gamma_8 (1 + gamma_8), rounded up
+    float absl;           // absolute slack
+    float big;            // max_h Q1_h * max(1, sum |w|): overflow guard
+    float pad[4];
+};
+static_assert(sizeof(QMeta) <= kQmBytes, "QMeta must fit its workspace slot");
+
+// ------------------------------------------------------------------------------------------------
+// Step 1: query terms.  One CTA per sequence, warp h = head h, lane l = dims 4l .. 4l+3.
+// qt[b] holds the shared-memory image of a 32-row x 128-byte K-major operand in the 128-byte
+// swizzle (row n at n*128, its 16-byte unit u at position u ^ (n & 7)): row 8i + h is term i of head
+// h, rows 24..31 are zero.  A plain copy into a 1024-byte-aligned buffer gives the MMA's layout.
+// ------------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) qterm_kernel(const uint16_t *__restrict__ iq, const float *__restrict__ iw,
+                                                    uint8_t *__restrict__ qt, QMeta *__restrict__ qm,
+                                                    int32_t *__restrict__ list_count, uint32_t *__restrict__ hist,
+                                                    uint32_t *__restrict__ hist2, uint32_t *__restrict__ seq_words)
+{
+    const int b = blockIdx.x, h = threadIdx.x >> 5, l = threadIdx.x & 31;
+    // the counters the later steps accumulate into start from zero on every call
+    if (b == 0 && threadIdx.x == 0 && list_count) *list_count = 0;
+    for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) {
+        hist[(size_t)b * kHistBins + i] = 0u;
+        if (hist2) hist2[(size_t)b * kHistBins + i] = 0u;
+    }
+    if (seq_words && threadIdx.x < kTopkWords) seq_words[(size_t)b * kTopkWords + threadIdx.x] = 0u;
+    const uint2 raw = reinterpret_cast<const uint2 *>(iq + ((size_t)b * kIdxHeads + h) * kIdxDim)[l];
+    const float q[4] = {bf16_lo(raw.x), bf16_hi(raw.x), bf16_lo(raw.y), bf16_hi(raw.y)};
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) amax = fmaxf(amax, fabsf(q[i]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    int s = 0;
+    if (amax > 0.f && amax <= 3.0e38f) {
+        int e;
+        frexpf(amax, &e);   // amax in [2^(e-1), 2^e)
+        s = 8 - e;          // scaled maximum in [128, 256)
+    }
+    uint32_t word[3] = {0u, 0u, 0u};
+    double t1 = 0.0, dl = 0.0, q1 = 0.0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float r = ldexpf(q[i], s);
+#pragma unroll
+        for (int term = 0; term < 3; ++term) {
+            const uint8_t c = (uint8_t)(f32x2_to_e4m3x2(r, 0.f) & 0xFF);
+            const float cv = e4m3_to_f32(c);
+            r = r - cv;   // exact: cv is r rounded to a coarser grid that r's own grid contains
+            t1 += fabs((double)cv);
+            word[term] |= (uint32_t)c << (8 * i);
+        }
+        dl += fabs((double)r);
+        q1 += fabs((double)q[i]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        t1 += __shfl_xor_sync(0xffffffffu, t1, o);
+        dl += __shfl_xor_sync(0xffffffffu, dl, o);
+        q1 += __shfl_xor_sync(0xffffffffu, q1, o);
+    }
+    uint8_t *img = qt + (size_t)b * kScrQtBytes;
+    const int d = 4 * l, unit = d >> 4, off = d & 15;
+#pragma unroll
+    for (int term = 0; term < 4; ++term) {
+        const int n = term * 8 + h;
+        *reinterpret_cast<uint32_t *>(img + n * 128 + ((unit ^ (n & 7)) << 4) + off) = term < 3 ? word[term] : 0u;
+    }
+    __shared__ double Fh[8], Q1h[8];
+    if (l == 0) {
+        const double inv = ldexp(1.0, -s);
+        Fh[h] = (kTcRel + gamma_n(2) * (1.0 + kTcRel)) * (t1 * inv) + dl * inv + gamma_n(19) * q1;
+        Q1h[h] = q1;
+        qm[b].inv_scale[h] = ldexpf(1.f, -s);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double G = 0.0, sw = 0.0, qmax = 0.0;
+        for (int hh = 0; hh < 8; ++hh) {
+            const double w = fabs((double)iw[(size_t)b * kIdxHeads + hh]);
+            G += w * Fh[hh];
+            sw += w;
+            qmax = fmax(qmax, Q1h[hh]);
+        }
+        const double g8 = gamma_n(8);
+        qm[b].G = (float)(G * (1.0 + g8) * kRoundUp);
+        qm[b].chain = (float)(2.0 * g8 * (1.0 + g8) * kRoundUp);
+        qm[b].absl = (float)(ldexp(1.0, -100) * (1.0 + sw) * 2.0);
+        qm[b].big = (float)(qmax * fmax(1.0, sw) * 1.01);   // NaN or inf when inputs are: no bounds
+    }
+}
+
+// ------------------------------------------------------------------------------------------------
+// Step 2: screen.  Persistent CTAs (one per SM), each taking a contiguous range of 128-position
+// tiles (two pages).  Warp 0 resolves tiles 32 at a time (one per lane) and issues the TMA loads of
+// their two key pages plus, when the sequence changed since that stage's last use, the query-term
+// image.  As soon as a stage lands, warp 1 issues the four K=32 MMAs of its tile into one of six
+// 32-column TMEM accumulators and one of two row-max groups (warps 2-5, 6-9; thread = row) writes
+// each row's largest |key| beside that accumulator; the stage is then free again (the MMA's commit
+// and the 128 row-max threads release it), so nearly all stages stay in flight.  Two groups of four epilogue warps (thread =
+// tile row = TMEM lane) take the tiles in turn (tile k: accumulator k mod 6, group k mod 2) and
+// turn accumulator and row maxima into per-block bounds.
+// ------------------------------------------------------------------------------------------------
+struct ScreenArgs {
+    const int32_t *seq_len;
+    const int32_t *block_table;
+    int max_pages;
+    int max_seq_len;
+    int B;
+    int num_pages;
+    int tiles_per_seq;
+    long long total;      // B * tiles_per_seq
+    long long per_cta;    // tiles per CTA
+    const float *iw;
+    const uint8_t *qt;
+    const QMeta *qm;
+    float *lo;
+    float *hi;
+    int stride;
+    uint32_t *hist;   // [B][kHistBins]: count of blocks per top 12 bits of the lower-bound key
+    void *ws;
+};
+
+struct ScrItem {
+    int b, L, tile;
+    int p0, p1;   // page ids of the tile's two pages (-1: none)
+};
+
+struct ScrSmem {
+    uint8_t keys[kScrStages][kScrKeyBytes];
+    uint8_t qt[kScrStages][kScrQtBytes];
+    float kmax[kScrAcc][kScrRows];   // largest |key| of each row, beside its accumulator
+    ScrItem ring[kScrRing];
+    uint64_t full[kScrStages], sfree[kScrStages], dfull[kScrAcc], dfree[kScrAcc], mma_fin;
+    int stage_b[kScrStages];
+    uint32_t tmem;
+    int abort_flag;
+};
+
+// kind::f8f6f4 instruction descriptor: D f32, A and B E4M3 (format 0), both K-major, M=128, N=32.
+constexpr uint32_t kIdescScreen =
+    (1u << 4) | ((uint32_t)(kScrN >> 3) << 17) | ((uint32_t)(kScrRows >> 4) << 24);
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+            "r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_mma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate)
+{
+    asm volatile(
+        "{\n.reg .pred p;\n"
+        "setp.ne.b32 p, %4, 0;\n"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Per 16-bit lane maximum of two words (sm_90+ SIMD integer max).
+__device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// Largest E4M3 magnitude code (bits 0-6) of a 128-byte key row in shared memory.  The row is in
+// the 128-byte swizzle, so thread r reads its 16-byte units in the order u ^ (r & 7), which spreads
+// the 8 threads of a quarter-warp over all 32 banks.  Magnitude codes order like the values they
+// encode.  Odd bytes are the high bytes of the 16-bit lanes of the masked words; even bytes become
+// high bytes after a shift by 8; a 16-bit max then keeps each high-byte maximum.
+__device__ __forceinline__ uint32_t row_max_code(const uint8_t *row, int r)
+{
+    const uint4 *p = reinterpret_cast<const uint4 *>(row);
+    uint32_t hi[8], lo[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {   // per 16-byte unit: a 2-level tree over its 4 words
+        const uint4 v = p[u ^ (r & 7)];
+        const uint32_t w0 = v.x & 0x7F7F7F7Fu, w1 = v.y & 0x7F7F7F7Fu, w2 = v.z & 0x7F7F7F7Fu, w3 = v.w & 0x7F7F7F7Fu;
+        hi[u] = vmax_u16x2(vmax_u16x2(w0, w1), vmax_u16x2(w2, w3));
+        lo[u] = vmax_u16x2(vmax_u16x2(w0 << 8, w1 << 8), vmax_u16x2(w2 << 8, w3 << 8));
+    }
+#pragma unroll
+    for (int s = 4; s > 0; s >>= 1)   // then a 3-level tree over the units
+#pragma unroll
+        for (int u = 0; u < s; ++u) {
+            hi[u] = vmax_u16x2(hi[u], hi[u + s]);
+            lo[u] = vmax_u16x2(lo[u], lo[u + s]);
+        }
+    return max(max(hi[0] >> 24, (hi[0] >> 8) & 0xFFu), max(lo[0] >> 24, (lo[0] >> 8) & 0xFFu));
+}
+
+__device__ __forceinline__ float no_lower() { return __uint_as_float(0xFFFFFFFFu); }   // -NaN: orders first
+__device__ __forceinline__ float no_upper() { return __uint_as_float(0x7FFFFFFFu); }   // +NaN: orders last
+
+__global__ void __launch_bounds__(kScrThreads, 1) screen_kernel(const __grid_constant__ CUtensorMap tmap,
+                                                                const ScreenArgs a)
+{
+    extern __shared__ uint8_t scr_raw[];
+    ScrSmem &sm = *reinterpret_cast<ScrSmem *>((reinterpret_cast<uintptr_t>(scr_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long first = (long long)blockIdx.x * a.per_cta;
+    const long long last = first + a.per_cta < a.total ? first + a.per_cta : a.total;
+    const long long n_items = last > first ? last - first : 0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kScrStages; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.sfree[s], 1 + 128);   // the MMA's commit and the row-max threads
+            sm.stage_b[s] = -1;
+        }
+        for (int d = 0; d < kScrAcc; ++d) {
+            mbar_init(&sm.dfull[d], 1 + 128);   // the MMA's commit and the row-max threads
+            mbar_init(&sm.dfree[d], 128);       // the epilogue group of accumulator d
+        }
+        mbar_init(&sm.mma_fin, 1);
+        sm.abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tc_alloc(smem_addr(&sm.tmem), kScrTmemCols);
+        tc_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem;
+
+    if (warp == 0) {
+        // ---------------- loader ----------------
+        auto resolve32 = [&](long long k0) {
+            const long long k = k0 + lane;
+            ScrItem it{-1, 0, 0, -1, -1};
+            if (k < n_items) {
+                const long long item = first + k;
+                const int b = (int)(item / a.tiles_per_seq), tile = (int)(item % a.tiles_per_seq);
+                const int L = a.seq_len[b];
+                it.b = b;
+                it.L = L;
+                it.tile = tile;
+                if (L < 1 || L > a.max_seq_len) {
+                    if (tile == 0) report(a.ws, CSA_ERR_DEVICE_DATA, b);
+                } else if (tile * kScrRows < L) {
+                    const int pg = 2 * tile;
+                    const int p0 = a.block_table[(size_t)b * a.max_pages + pg];
+                    if (p0 < 0 || p0 >= a.num_pages) {
+                        report(a.ws, CSA_ERR_DEVICE_DATA, (long long)b * a.max_pages + pg);
+                    } else {
+                        it.p0 = p0;
+                        if ((pg + 1) * kPage < L) {
+                            const int p1 = a.block_table[(size_t)b * a.max_pages + pg + 1];
+                            if (p1 < 0 || p1 >= a.num_pages) {
+                                report(a.ws, CSA_ERR_DEVICE_DATA, (long long)b * a.max_pages + pg + 1);
+                                it.p0 = -1;
+                            } else {
+                                it.p1 = p1;
+                            }
+                        }
+                    }
+                }
+            }
+            sm.ring[k % kScrRing] = it;
+        };
+        long long issued = 0;
+        for (long long k = 0; k < n_items; ++k) {
+            if ((k & 31) == 0) {
+                resolve32(k);
+                __syncwarp();
+            }
+            const int st = (int)(k % kScrStages);
+            int ok = 1;
+            if (lane == 0) {
+                ok = mbar_wait(&sm.sfree[st], (uint32_t)(((k / kScrStages) & 1) ^ 1), &sm.abort_flag, a.ws, 20) ? 1 : 0;
+                if (ok) {
+                    const ScrItem it = sm.ring[k % kScrRing];
+                    if (it.p0 >= 0) {
+                        const bool need_q = sm.stage_b[st] != it.b;
+                        const uint32_t bytes = (it.p1 >= 0 ? kScrKeyBytes : kScrPageBytes) + (need_q ? kScrQtBytes : 0u);
+                        mbar_arrive_expect_tx(&sm.full[st], bytes);
+                        tma_load_2d(sm.keys[st], &tmap, 0, it.p0 * kPage, &sm.full[st]);
+                        if (it.p1 >= 0) tma_load_2d(sm.keys[st] + kScrPageBytes, &tmap, 0, it.p1 * kPage, &sm.full[st]);
+                        if (need_q) {
+                            bulk_g2s(sm.qt[st], a.qt + (size_t)it.b * kScrQtBytes, kScrQtBytes, &sm.full[st]);
+                            sm.stage_b[st] = it.b;
+                        }
+                    } else {
+                        mbar_arrive(&sm.full[st]);
+                    }
+                }
+            }
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            issued = k + 1;
+        }
+        // no copy may still be landing in shared memory when the CTA exits
+        if (lane == 0) {
+            for (long long kk = issued > kScrStages ? issued - kScrStages : 0; kk < issued; ++kk) {
+                volatile int no_abort = 0;
+                mbar_wait(&sm.full[kk % kScrStages], (uint32_t)((kk / kScrStages) & 1), &no_abort, a.ws, 25);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            bool any_mma = false;
+            for (long long k = 0; k < n_items; ++k) {
+                const int st = (int)(k % kScrStages), d = (int)(k % kScrAcc);
+                if (!mbar_wait(&sm.full[st], (uint32_t)((k / kScrStages) & 1), &sm.abort_flag, a.ws, 21)) break;
+                if (!mbar_wait(&sm.dfree[d], (uint32_t)(((k / kScrAcc) & 1) ^ 1), &sm.abort_flag, a.ws, 22)) break;
+                tc_fence_after();
+                if (sm.ring[k % kScrRing].p0 >= 0) {
+                    const uint32_t ka = smem_addr(sm.keys[st]), kb = smem_addr(sm.qt[st]);
+#pragma unroll
+                    for (int kk = 0; kk < kIdxDim / 32; ++kk)
+                        tc_mma_f8(tmem + 32 * d, umma_sdesc_sw128(ka + kk * 32, 16, 1024),
+                                  umma_sdesc_sw128(kb + kk * 32, 16, 1024), kIdescScreen, kk > 0);
+                    tc_commit(smem_addr(&sm.dfull[d]));
+                    tc_commit(smem_addr(&sm.sfree[st]));
+                    any_mma = true;
+                } else {
+                    mbar_arrive(&sm.dfull[d]);
+                    mbar_arrive(&sm.sfree[st]);
+                }
+            }
+            if (any_mma) {   // every MMA this thread issued has finished before TMEM is released
+                tc_commit(smem_addr(&sm.mma_fin));
+                volatile int no_abort = 0;
+                mbar_wait(&sm.mma_fin, 0, &no_abort, a.ws, 26);
+            }
+        }
+        __syncwarp();
+    } else if (warp < kScrEpiWarp0) {
+        // ---------------- row maxima, group mg: tiles k = mg, mg + 2, ...; thread = tile row ----------
+        const int mg = (warp - 2) >> 2;
+        const int r = threadIdx.x - 64 - 128 * mg;
+        for (long long k = mg; k < n_items; k += kScrMaxGroups) {
+            const int st = (int)(k % kScrStages), d = (int)(k % kScrAcc);
+            if (!warp_wait(&sm.full[st], (uint32_t)((k / kScrStages) & 1), &sm.abort_flag, a.ws, 27)) break;
+            if (!warp_wait(&sm.dfree[d], (uint32_t)(((k / kScrAcc) & 1) ^ 1), &sm.abort_flag, a.ws, 28)) break;
+            if (sm.ring[k % kScrRing].p0 >= 0)
+                sm.kmax[d][r] = e4m3_to_f32((uint8_t)row_max_code(sm.keys[st] + r * kIdxDim, r));
+            mbar_arrive(&sm.dfull[d]);
+            mbar_arrive(&sm.sfree[st]);
+        }
+    } else {
+        // ---------------- epilogue group g: tiles k = g, g + 2, ...; thread = tile row = TMEM lane ----
+        const int g = (warp - kScrEpiWarp0) >> 2;
+        const int quad = warp & 3;
+        const int r = 32 * quad + lane;
+        const uint32_t tl = tmem + ((uint32_t)(32 * quad) << 16);
+        int cur_b = -1;
+        QMeta qm{};
+        float w[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (long long k = g; k < n_items; k += kScrEpiGroups) {
+            const int d = (int)(k % kScrAcc);
+            if (!warp_wait(&sm.dfull[d], (uint32_t)((k / kScrAcc) & 1), &sm.abort_flag, a.ws, 24)) break;
+            tc_fence_after();
+            const ScrItem it = sm.ring[k % kScrRing];
+            if (it.p0 >= 0) {
+                if (it.b != cur_b) {
+                    cur_b = it.b;
+                    qm = a.qm[it.b];
+#pragma unroll
+                    for (int h = 0; h < 8; ++h) w[h] = a.iw[(size_t)it.b * kIdxHeads + h];
+                }
+                const float kmax = sm.kmax[d][r];
+                float D[32];
+                tc_ld32_sync(tl + 32 * d, D);
+                float t = 0.f, wr = 0.f;
+#pragma unroll
+                for (int h = 0; h < 8; ++h) {
+                    const float dh = __fmul_rn(__fadd_rn(__fadd_rn(D[h], D[8 + h]), D[16 + h]), qm.inv_scale[h]);
+                    const float rh = dh > 0.f ? dh : 0.f;
+                    t = __fmaf_rn(w[h], rh, t);
+                    wr = __fmaf_ru(fabsf(w[h]), rh, wr);
+                }
+                const float eps = __fmaf_ru(kmax, qm.G, __fmaf_ru(qm.chain, wr, qm.absl));
+                float lo, hi;
+                const int p = it.tile * kScrRows + r;
+                if (p >= it.L) {
+                    lo = -INFINITY;   // not a position: leaves the block's maxima alone
+                    hi = -INFINITY;
+                } else if (!(__fmul_ru(kmax, qm.big) < 1e37f) || !(fabsf(t) <= 3.0e38f) || !(eps <= 3.0e38f)) {
+                    lo = no_lower();
+                    hi = no_upper();
+                } else {
+                    lo = __fsub_rd(t, eps);
+                    hi = __fadd_ru(t, eps);
+                }
+                // block = 8 consecutive rows = 8 consecutive lanes.  The block score is the max of its
+                // positions' scores, so the max of their lower bounds and the max of their upper bounds
+                // bound it (a position without bounds has the smallest lower and largest upper key).
+                uint32_t klo = order_key(lo), khi = order_key(hi);
+#pragma unroll
+                for (int o = 1; o < 8; o <<= 1) {
+                    klo = max(klo, __shfl_xor_sync(0xffffffffu, klo, o));
+                    khi = max(khi, __shfl_xor_sync(0xffffffffu, khi, o));
+                }
+                const int blk = it.tile * (kScrRows / kBlock) + r / kBlock;
+                if ((lane & 7) == 0 && blk * kBlock < it.L) {
+                    const size_t o = (size_t)it.b * a.stride + blk;
+                    a.lo[o] = __uint_as_float(klo & 0x80000000u ? klo & 0x7FFFFFFFu : ~klo);
+                    a.hi[o] = __uint_as_float(khi & 0x80000000u ? khi & 0x7FFFFFFFu : ~khi);
+                    atomicAdd(&a.hist[(size_t)it.b * kHistBins + (klo >> 20)], 1u);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&sm.dfree[d]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tc_dealloc(tmem, kScrTmemCols);
+}
+
+// ------------------------------------------------------------------------------------------------
+// Step 3: classification, over a grid of (chunk, sequence) CTAs.  With T <= the k-th largest lower
+// bound and U >= the (k+1)-th largest upper bound, a block is
+//   out        if upper < T: k blocks have lower >= T, so k scores are >= T, above this one's;
+//   sure       if lower > U: only blocks with upper > U, at most k of them and this block among
+//              them, can reach its score, so it is in the Top-K whatever the ties;
+//   uncertain  otherwise: scored exactly afterwards.
+// The k-th largest lower-bound key X is located to 24 bits: its top 12 bits from the screen's
+// per-sequence histogram, the next 12 from a second histogram of the keys in that bin (pass A).
+// T = X with the last 8 bits clear; U = (X with them set) + the widest interval of the sequence,
+// rounded up (pass A takes that maximum too): a block with upper > U has lower > X, and fewer than k
+// blocks do.  If some bound of the sequence is not finite, U is the largest key: no block is sure.
+// Pass B writes every block's class and appends the uncertain blocks to the sequence's slice and to
+// the global re-scoring work list.
+// ------------------------------------------------------------------------------------------------
+constexpr int kClsThreads = 256;
+constexpr uint8_t kOut = 0, kSure = 1, kUncertain = 2, kChosen = 3, kTie = 4;
+
+// Per-sequence words: [0] sure blocks, [1] uncertain blocks, [2] order key of the widest interval.
+struct SeqWords {
+    uint32_t n_sure, n_uncertain, wmax_key, pad;
+};
+static_assert(sizeof(SeqWords) == kTopkWords * 4, "SeqWords fills one sequence's select words");
+
+__device__ __forceinline__ float key_to_float(uint32_t u)
+{
+    return __uint_as_float((u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u);
+}
+
+// Over a kHistBins-bin histogram h: the bin holding the rank-th largest element (1-based) and that
+// element's rank inside the bin; every thread gets both.  If the counts fall short of rank: bin 0
+// (a threshold that keeps everything).
+template <int kThreads>
+__device__ __forceinline__ void rank_bin(const uint32_t *h, uint32_t rank, uint32_t *scratch, int *bin_out,
+                                         uint32_t *rank_out)
+{
+    constexpr int kPer = kHistBins / kThreads;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    if (t == 0) {
+        scratch[33] = 0u;
+        scratch[34] = 1u;
+    }
+    // thread t owns the kPer bins below kHistBins - kPer t, largest first
+    uint32_t c[kPer], s = 0;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+        c[i] = h[kHistBins - 1 - kPer * t - i];
+        s += c[i];
+    }
+    uint32_t x = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) scratch[warp] = x;
+    __syncthreads();
+    uint32_t before = 0;
+    for (int wi = 0; wi < warp; ++wi) before += scratch[wi];
+    uint32_t run = before + x - s;   // elements in larger bins than this thread's
+    if (run < rank && rank <= run + s) {
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            if (run < rank && rank <= run + c[i]) {
+                scratch[33] = (uint32_t)(kHistBins - 1 - kPer * t - i);
+                scratch[34] = rank - run;
+            }
+            run += c[i];
+        }
+    }
+    __syncthreads();
+    *bin_out = (int)scratch[33];
+    *rank_out = scratch[34];
+    __syncthreads();
+}
+
+struct ClsArgs {
+    const float *lo;
+    const float *hi;
+    int stride;          // row stride of lo, hi and uslice (blocks)
+    int sstride;         // row stride of status (bytes, a multiple of 16)
+    const int32_t *seq_len;
+    int max_seq_len;
+    int k;
+    const uint32_t *hist;
+    uint32_t *hist2;
+    SeqWords *words;
+    uint8_t *status;
+    int32_t *uslice;
+    uint2 *list;
+    int32_t *list_count;
+    void *ws;
+};
+
+__device__ __forceinline__ bool cls_chunk(const ClsArgs &a, int b, int &n, int &i0, int &i1)
+{
+    const int L = a.seq_len[b];
+    if (L < 1 || L > a.max_seq_len) return false;
+    n = (L + kBlock - 1) / kBlock;
+    if (n <= a.k) return false;   // every block is selected
+    const int per = (n + gridDim.x - 1) / gridDim.x;
+    i0 = blockIdx.x * per;
+    i1 = min(n, i0 + per);
+    return i0 < i1;
+}
+
+__global__ void __launch_bounds__(kClsThreads) classify_a_kernel(const ClsArgs a)
+{
+    __shared__ uint32_t scratch[40];
+    const int b = blockIdx.y;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        const int L = a.seq_len[b];
+        if (L < 1 || L > a.max_seq_len) report(a.ws, CSA_ERR_DEVICE_DATA, b);
+    }
+    int n, i0, i1;
+    if (!cls_chunk(a, b, n, i0, i1)) return;
+    int bin1;
+    uint32_t r1;
+    rank_bin<kClsThreads>(a.hist + (size_t)b * kHistBins, (uint32_t)a.k, scratch, &bin1, &r1);
+    const float *lp = a.lo + (size_t)b * a.stride;
+    const float *hp = a.hi + (size_t)b * a.stride;
+    uint32_t *h2 = a.hist2 + (size_t)b * kHistBins;
+    uint32_t wkey = 0u;   // order key of the widest interval (+inf when a bound is not finite)
+    for (int i = i0 + threadIdx.x; i < i1; i += kClsThreads) {
+        const float l = lp[i], h = hp[i];
+        const float w = __fsub_ru(h, l);
+        wkey = max(wkey, w == w ? order_key(w) : 0xFF800000u);
+        const uint32_t kl = order_key(l);
+        if ((int)(kl >> 20) == bin1) atomicAdd(&h2[(kl >> 8) & (kHistBins - 1)], 1u);
+    }
+    wkey = block_reduce_minmax(wkey, true, scratch);
+    if (threadIdx.x == 0) atomicMax(&a.words[b].wmax_key, wkey);
+}
+
+__global__ void __launch_bounds__(kClsThreads) classify_b_kernel(const ClsArgs a)
+{
+    __shared__ uint32_t scratch[40];
+    const int b = blockIdx.y, lane = threadIdx.x & 31;
+    int n, i0, i1;
+    if (!cls_chunk(a, b, n, i0, i1)) return;
+    int bin1, bin2;
+    uint32_t r1, r2;
+    rank_bin<kClsThreads>(a.hist + (size_t)b * kHistBins, (uint32_t)a.k, scratch, &bin1, &r1);
+    rank_bin<kClsThreads>(a.hist2 + (size_t)b * kHistBins, r1, scratch, &bin2, &r2);
+    const uint32_t T = ((uint32_t)bin1 << 20) | ((uint32_t)bin2 << 8);
+    const uint32_t wkey = a.words[b].wmax_key;
+    const float wmax = key_to_float(wkey);
+    const uint32_t U = wkey >= 0xFF800000u ? 0xFFFFFFFFu : order_key(__fadd_ru(key_to_float(T | 0xFFu), wmax));
+    const float *lp = a.lo + (size_t)b * a.stride;
+    const float *hp = a.hi + (size_t)b * a.stride;
+    uint8_t *stat = a.status + (size_t)b * a.sstride;
+    int32_t *us = a.uslice + (size_t)b * a.stride;
+    const uint32_t lt = (1u << lane) - 1u;
+    uint32_t n_sure = 0;
+    for (int base = i0 + (threadIdx.x & ~31); base < i1; base += kClsThreads) {
+        const int i = base + lane;
+        uint8_t c = kOut;
+        if (i < i1) {
+            const uint32_t hk = order_key(hp[i]), lk = order_key(lp[i]);
+            c = hk < T ? kOut : (lk > U ? kSure : kUncertain);
+            stat[i] = c;
+        }
+        n_sure += c == kSure;
+        // uncertain blocks: one atomic per warp for the slice and one for the work list
+        const uint32_t bu = __ballot_sync(0xffffffffu, c == kUncertain);
+        if (bu) {
+            uint32_t sbase = 0, lbase = 0;
+            if (lane == 0) {
+                sbase = atomicAdd(&a.words[b].n_uncertain, (uint32_t)__popc(bu));
+                lbase = (uint32_t)atomicAdd(a.list_count, __popc(bu));
+            }
+            sbase = __shfl_sync(0xffffffffu, sbase, 0);
+            lbase = __shfl_sync(0xffffffffu, lbase, 0);
+            if (c == kUncertain) {
+                const uint32_t r = __popc(bu & lt);
+                us[sbase + r] = i;
+                a.list[lbase + r] = make_uint2((uint32_t)b, (uint32_t)i);
+            }
+        }
+    }
+    n_sure = block_reduce_sum(n_sure, scratch);
+    if (threadIdx.x == 0 && n_sure) atomicAdd(&a.words[b].n_sure, n_sure);
+}
+
+// ------------------------------------------------------------------------------------------------
+// Step 5 (after the exact re-scoring of the uncertain blocks): the sure blocks plus the
+// k - n_sure best uncertain ones by exact score (larger first, then lower block id), written in
+// ascending block order.  One CTA per sequence.  The chosen uncertain blocks are found on the
+// sequence's slice -- by counting each one's rank when there are few, else by radix selection, whose
+// blocks tied at the threshold are marked and the lowest-numbered need_eq of them taken -- and marked
+// in the status bytes; one ordered pass over the status bytes writes the result.
+// ------------------------------------------------------------------------------------------------
+constexpr int kFinThreads = 1024;
+constexpr int kFinWarps = kFinThreads / 32;
+constexpr int kFinCache = 16384;         // uncertain keys cached up to this many
+constexpr int kFinRankMax = 512;         // up to this many uncertain blocks: rank by counting
+constexpr int kFinStatusCache = 65536;   // status bytes staged in shared memory up to this many blocks
+
+__global__ void __launch_bounds__(kFinThreads, 1) finalize_kernel(
+    const float *__restrict__ scores, int score_stride, const int32_t *__restrict__ seq_len, int max_seq_len,
+    uint8_t *__restrict__ status, int sstride, const int32_t *__restrict__ uslice, const SeqWords *__restrict__ words,
+    int stride, int k, int32_t *__restrict__ out_blocks, int32_t *__restrict__ out_count, void *ws)
+{
+    extern __shared__ uint32_t fz_smem[];
+    uint32_t *whist = fz_smem;                    // [32 warps][256]
+    uint32_t *skeys = whist + kFinWarps * 256;    // keys of the uncertain blocks
+    int32_t *sblk = reinterpret_cast<int32_t *>(skeys + kFinRankMax);   // their ids (rank path)
+    uint8_t *sstat = reinterpret_cast<uint8_t *>(skeys + kFinCache);    // staged status bytes
+    __shared__ uint32_t scratch[72];
+    __shared__ uint32_t sel[2];
+    const int b = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int L = seq_len[b];
+    int32_t *out = out_blocks + (size_t)b * k;
+    if (L < 1 || L > max_seq_len) {   // reported by the classification
+        if (t == 0) out_count[b] = 0;
+        return;
+    }
+    const int n = (L + kBlock - 1) / kBlock;
+    if (n <= k) {   // every block is selected
+        for (int i = t; i < n; i += kFinThreads) out[i] = i;
+        if (t == 0) out_count[b] = n;
+        return;
+    }
+    const SeqWords sw = words[b];
+    const int n_sure = (int)sw.n_sure, nu = (int)sw.n_uncertain;
+    const int kk = k - n_sure;   // how many uncertain blocks to take
+    if (n_sure > k || kk > nu) {
+        if (t == 0) {
+            out_count[b] = 0;
+            report(ws, CSA_ERR_DEVICE_DATA, (long long)b);
+        }
+        return;
+    }
+    const float *sc = scores + (size_t)b * score_stride;
+    const int32_t *us = uslice + (size_t)b * stride;
+    uint8_t *stat = status + (size_t)b * sstride;
+    const bool staged = n <= kFinStatusCache;
+    if (staged) {   // status row into shared memory, 16 bytes per load
+        const int nv = (n + 15) >> 4;
+        for (int i = t; i < nv; i += kFinThreads)
+            reinterpret_cast<uint4 *>(sstat)[i] = reinterpret_cast<const uint4 *>(stat)[i];
+    }
+    uint8_t *st8 = staged ? sstat : stat;
+    uint32_t need_eq = 0;
+    if (kk > 0 && kk == nu) {
+        __syncthreads();
+        for (int j = t; j < nu; j += kFinThreads) st8[us[j]] = kChosen;
+    } else if (kk > 0 && nu <= kFinRankMax) {
+        for (int j = t; j < nu; j += kFinThreads) {
+            const int blk = us[j];
+            sblk[j] = blk;
+            skeys[j] = order_key(sc[blk]);
+        }
+        __syncthreads();
+        // warp per uncertain block, its lanes splitting the comparisons
+        for (int j = warp; j < nu; j += kFinWarps) {
+            const uint32_t u = skeys[j];
+            const int bj = sblk[j];
+            int rank = 0;
+            for (int i = lane; i < nu; i += 32) {
+                const uint32_t x = skeys[i];
+                rank += (x > u) || (x == u && sblk[i] < bj);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) rank += __shfl_xor_sync(0xffffffffu, rank, o);
+            if (lane == 0 && rank < kk) st8[bj] = kChosen;
+        }
+    } else if (kk > 0) {
+        const bool cached = nu <= kFinCache;
+        if (cached)
+            for (int j = t; j < nu; j += kFinThreads) skeys[j] = order_key(sc[us[j]]);
+        __syncthreads();
+        auto key = [&](int j) { return cached ? skeys[j] : order_key(sc[us[j]]); };
+        uint32_t T;
+        radix_select<kFinThreads>(nu, (uint32_t)kk, key, 0, whist, scratch, sel, T, need_eq);
+        for (int j = t; j < nu; j += kFinThreads) {
+            const uint32_t u = key(j);
+            if (u > T) st8[us[j]] = kChosen;
+            else if (u == T) st8[us[j]] = kTie;
+        }
+    } else {
+        __syncthreads();
+    }
+    __syncthreads();
+    // ordered output: sure and chosen blocks, and the first need_eq tied ones.  Thread t owns the
+    // bytes [t c, t c + c), c a multiple of 16, read 16 at a time.
+    const int c = ((n + kFinThreads - 1) / kFinThreads + 15) & ~15;
+    const int i0 = min(n, t * c), i1 = min(n, i0 + c);
+    auto cls = [](uint32_t v, int j) { return (v >> (8 * j)) & 0xFFu; };
+    uint32_t n_take = 0, n_tie = 0;
+    for (int i = i0; i < i1; i += 16) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(st8 + i);
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+            const uint32_t x = cls(w4[q >> 2], q & 3);
+            const bool in = i + q < i1;
+            n_take += in && (x == kSure || x == kChosen);
+            n_tie += in && x == kTie;
+        }
+    }
+    // exclusive scan of (n_take, n_tie) over the CTA
+    uint32_t x = n_take, y = n_tie;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t xa = __shfl_up_sync(0xffffffffu, x, o), ya = __shfl_up_sync(0xffffffffu, y, o);
+        if (lane >= o) {
+            x += xa;
+            y += ya;
+        }
+    }
+    if (lane == 31) {
+        scratch[warp] = x;
+        scratch[32 + warp] = y;
+    }
+    __syncthreads();
+    uint32_t r_take = x - n_take, r_tie = y - n_tie, total = 0, total_tie = 0;
+    for (int wi = 0; wi < kFinWarps; ++wi) {
+        const uint32_t a0 = scratch[wi], a1 = scratch[32 + wi];
+        if (wi < warp) {
+            r_take += a0;
+            r_tie += a1;
+        }
+        total += a0;
+        total_tie += a1;
+    }
+    for (int i = i0; i < i1; i += 16) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(st8 + i);
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+            if (i + q >= i1) break;
+            const uint32_t xq = cls(w4[q >> 2], q & 3);
+            if (xq == kSure || xq == kChosen) {
+                const uint32_t pos = r_take + min(r_tie, need_eq);
+                if (pos < (uint32_t)k) out[pos] = i + q;
+                ++r_take;
+            } else if (xq == kTie) {
+                if (r_tie < need_eq && r_take + r_tie < (uint32_t)k) out[r_take + r_tie] = i + q;
+                ++r_tie;
+            }
+        }
+    }
+    if (t == 0) {
+        out_count[b] = k;
+        if (total + min(total_tie, need_eq) != (uint32_t)k) report(ws, CSA_ERR_DEVICE_DATA, (long long)b);
+    }
+}
+
+// ------------------------------------------------------------------------------------------------
+// Host side
+// ------------------------------------------------------------------------------------------------
+namespace {
+
+std::mutex g_encode_mu;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+// The driver's tensor-map encoder, looked up once through the runtime (no link against libcuda).
+cudaError_t tensor_map_encoder(PFN_cuTensorMapEncodeTiled_v12000 *out)
+{
+    std::lock_guard<std::mutex> lock(g_encode_mu);
+    if (!g_encode) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        const cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+        if (e != cudaSuccess) return e;
+        if (q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    *out = g_encode;
+    return cudaSuccess;
+}
+
+int g_sm_count[64];
+
+int sm_count()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return kNumSms;
+    if (!g_sm_count[dev]) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        g_sm_count[dev] = n > 0 ? n : kNumSms;
+    }
+    return g_sm_count[dev];
+}
+
+}  // namespace
+
+// Keys as a 2-D tensor [num_pages * 64 rows][128 bytes], boxes of one page, 128-byte swizzle.
+bool screen_supported(int num_pages) { return (long long)num_pages * kPage <= 0xFFFFFFFFll; }
+
+cudaError_t launch_screen_bounds(const uint8_t *keys, int num_pages, const csa_batch &bt, const uint16_t *iq,
+                                 const float *iw, uint8_t *qt, void *qm, int32_t *list_count, uint32_t *hist,
+                                 uint32_t *hist2, void *words, float *lo, float *hi, int stride, void *ws,
+                                 cudaStream_t st)
+{
+    cudaError_t e;
+    PFN_cuTensorMapEncodeTiled_v12000 encode;
+    if ((e = tensor_map_encoder(&encode)) != cudaSuccess) return e;
+    CUtensorMap map;
+    const cuuint64_t dims[2] = {(cuuint64_t)kIdxDim, (cuuint64_t)num_pages * kPage};
+    const cuuint64_t strides[1] = {(cuuint64_t)kIdxDim};
+    const cuuint32_t box[2] = {(cuuint32_t)kIdxDim, (cuuint32_t)kPage};
+    const cuuint32_t estr[2] = {1, 1};
+    if (encode(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(keys), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+
+    qterm_kernel<<<bt.B, 256, 0, st>>>(iq, iw, qt, reinterpret_cast<QMeta *>(qm), list_count, hist, hist2,
+                                       reinterpret_cast<uint32_t *>(words));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+    ScreenArgs sa;
+    sa.seq_len = bt.seq_len;
+    sa.block_table = bt.block_table;
+    sa.max_pages = bt.max_pages;
+    sa.max_seq_len = bt.max_seq_len;
+    sa.B = bt.B;
+    sa.num_pages = num_pages;
+    sa.tiles_per_seq = (bt.max_seq_len + kScrRows - 1) / kScrRows;
+    sa.total = (long long)bt.B * sa.tiles_per_seq;
+    const int grid = (int)(sa.total < sm_count() ? sa.total : sm_count());
+    sa.per_cta = (sa.total + grid - 1) / grid;
+    sa.iw = iw;
+    sa.qt = qt;
+    sa.qm = reinterpret_cast<const QMeta *>(qm);
+    sa.lo = lo;
+    sa.hi = hi;
+    sa.stride = stride;
+    sa.hist = hist;
+    sa.ws = ws;
+    const size_t smem = sizeof(ScrSmem) + 1024;
+    if ((e = cudaFuncSetAttribute(screen_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+        return e;
+    screen_kernel<<<grid, kScrThreads, smem, st>>>(map, sa);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_classify(const float *lo, const float *hi, int stride, const csa_batch &bt, int k,
+                            const uint32_t *hist, uint32_t *hist2, void *words, uint8_t *status, int sstride,
+                            int32_t *uslice, uint2 *list, int32_t *list_count, void *ws, cudaStream_t st)
+{
+    ClsArgs a;
+    a.lo = lo;
+    a.hi = hi;
+    a.stride = stride;
+    a.sstride = sstride;
+    a.seq_len = bt.seq_len;
+    a.max_seq_len = bt.max_seq_len;
+    a.k = k;
+    a.hist = hist;
+    a.hist2 = hist2;
+    a.words = reinterpret_cast<SeqWords *>(words);
+    a.status = status;
+    a.uslice = uslice;
+    a.list = list;
+    a.list_count = list_count;
+    a.ws = ws;
+    // about two CTAs per SM over the batch, at least 512 blocks per chunk
+    const int nb = (bt.max_seq_len + kBlock - 1) / kBlock;
+    int chunks = (2 * sm_count() + bt.B - 1) / bt.B;
+    const int max_chunks = (nb + 511) / 512;
+    if (chunks > max_chunks) chunks = max_chunks;
+    if (chunks < 1) chunks = 1;
+    const dim3 grid(chunks, bt.B);
+    classify_a_kernel<<<grid, kClsThreads, 0, st>>>(a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    classify_b_kernel<<<grid, kClsThreads, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_finalize(const float *scores, int score_stride, const csa_batch &bt, uint8_t *status,
+                            int sstride, const int32_t *uslice, const void *words, int stride, int k,
+                            int32_t *out_blocks, int32_t *out_count, void *ws, cudaStream_t st)
+{
+    const size_t smem = ((size_t)kFinWarps * 256 + kFinCache) * 4 + kFinStatusCache;
+    static_assert(2 * kFinRankMax <= kFinCache, "rank-path keys and ids share the key cache");
+    cudaError_t e = cudaFuncSetAttribute(finalize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    finalize_kernel<<<bt.B, kFinThreads, smem, st>>>(scores, score_stride, bt.seq_len, bt.max_seq_len, status, sstride,
+                                                      uslice, reinterpret_cast<const SeqWords *>(words), stride, k,
+                                                      out_blocks, out_count, ws);
+    return cudaGetLastError();
+}
+
+}  // namespace csa

@@ -130,10 +130,31 @@ csa_status csa_kv_pack_fp4(const csa_kv_layer *layer, const uint16_t *latent,
  * per head, eight 16-dim FMA chains part_j, then ((p0+p4)+(p2+p6)) + ((p1+p5)+(p3+p7)), ReLU, and
  * an FMA chain over h = 0..7.  Block score = max over its positions < seq_len.  Order: larger
  * score first, then lower block id.  The selected set is bit-for-bit defined.
+ * How: every position is first screened on the tensor cores (csa_indexer_screen_bounds); only
+ * the blocks whose upper bound reaches the k-th largest lower bound are scored exactly, which
+ * provably contains the exact Top-k, so the result equals an exhaustive exact scan.  ws: at least
+ * csa_workspace_bytes(B, any H, max_seq_len, k) bytes.
  */
 csa_status csa_indexer_full(const csa_kv_layer *layer, const csa_batch *batch, const uint16_t *iq,
                             const float *iw, int32_t k, int32_t *out_blocks, int32_t *out_count,
                             void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Screening bounds of the Full-layer score (no counterpart in the pages: this exposes the first
+ * stage of csa_indexer_full for checking).  For every block v < ceil(seq_len/8) of every sequence,
+ *   lower[b][v] <= exact block score <= upper[b][v]
+ * in the order Top-K uses (a total order on binary32 with -0 = +0, NaN with the sign bit clear above
+ * +inf and with it set below -inf).  A block whose bound cannot be formed (non-finite inputs, or
+ * magnitudes near binary32 overflow) gets lower = -NaN and upper = +NaN, the two ends of that order.
+ * The approximate score comes from E4M3 x E4M3 tensor-core products of the keys with a 3-term E4M3
+ * split of q; the half-width is a rigorous bound on its distance to the exact binary32 chain.
+ *   lower, upper float [B][stride], stride >= ceil(max_seq_len/8); entries past each row's count are
+ *   untouched.  ws: csa_workspace_bytes(B, any H, max_seq_len, 1) bytes.
+ * Returns CSA_ERR_UNSUPPORTED if num_pages * 64 >= 2^32 (the keys' tensor-map limit).
+ */
+csa_status csa_indexer_screen_bounds(const csa_kv_layer *layer, const csa_batch *batch,
+                                     const uint16_t *iq, const float *iw, float *lower, float *upper,
+                                     int32_t stride, void *ws, size_t ws_bytes, void *stream);
 
 /*
  * Steps 2-3, Reindex layer -- re-score only the pool's blocks with this layer's own query and
