@@ -6,10 +6,11 @@
 // the kernel, in parallel).  The 512-channel latent serves as both key and value.
 //
 // With 64 heads sharing one latent, QK^T and PV are dense contractions: 4 x 64 x 512 FLOP per 288-B
-// entry, above the fp16 tensor ridge of B200, so they run on the tensor cores.  Dequantisation is
-// exact in fp16 (an E2M1 value times an E4M3 scale has at most 6 significant bits and lies in
-// [2^-10, 2688]); Q is scaled per head by a power of two into fp16's range; P is rounded to fp16
-// (relative error 2^-11); accumulation is fp32 in TMEM.
+// entry, above the fp16 tensor ridge of B200, so they run on the tensor cores.  Dequantisation of
+// the FP4 entries is exact in fp16 (an E2M1 value times an E4M3 scale has at most 6 significant bits
+// and lies in [2^-10, 2688]); a window entry's E4M3 values times its binary32 scale are rounded to
+// fp16 (relative error 2^-11); Q is scaled per head by a power of two into fp16's range; P is rounded
+// to fp16 (relative error 2^-11); accumulation is fp32 in TMEM.
 //
 // Tile = 128 entries.  Both MMAs put the entries / channels on M = 128 ("swap AB"):
 //   QK:  S^T[128 entries x 64 heads]  = V[128 x 512] . Q^T          (A = V K-major, B = Q K-major)
@@ -18,18 +19,20 @@
 // so TMEM holds S^T in 64 columns, O^T in 256 and L^T in 64, and one 128-byte-swizzled fp16 copy of
 // the tile in shared memory is read as K-major V by QK and as MN-major V^T by PV.  The all-ones
 // operand is one 128-byte block read through a zero-stride descriptor; summing the same fp16 P on the
-// tensor core keeps the normaliser consistent with the numerator.  Window rows carry their FP8 scale
-// in P (so PV multiplies by it); their sum is corrected by p * (1 - scale) in shared memory.
+// tensor core keeps the normaliser consistent with the numerator.
 //
 // Warp roles (288 threads).  Warp 8 owns the TMEM allocation and its lane 0 issues every MMA: QK of
 // tile t chunk by chunk as its 64-channel chunks are dequantised, then PV and L of tile t once P is
-// in shared memory.  Group 1 = warps 0-3 (TMEM lanes 0-127) runs the softmax and the epilogue.
-// Group 0 = warps 4-7 loads Q once and writes each tile's entry metadata.  Both groups dequantise:
-// thread e of a group takes tile row e and the group's four 64-channel chunks (0, 1, 4, 5 for group
-// 0; 2, 3, 6, 7 for group 1) from raw entries prefetched into registers a tile ahead.  The V buffer
-// is single; the chunks of tile t+1 are written as soon as PV(t) has finished the M-tile reading
-// them, so dequantisation and the QK of tile t+1 overlap the end of PV(t).  Softmax rescales lazily:
-// O^T and L^T are rescaled in TMEM only when a head's running maximum grows by more than 2^8.
+// in shared memory.  Warps 0-7 form two groups of four (TMEM lanes 0-127 each; thread = tile row):
+// group 1 = warps 0-3 takes heads 0-31 of the softmax and the epilogue, group 0 = warps 4-7 heads
+// 32-63 and also writes each tile's entry metadata; the two halves are independent, each with its own
+// named barrier.  Both groups load Q and dequantise: thread e of a group takes tile row e and the
+// group's four 64-channel chunks (0, 1, 4, 5 for group 0; 2, 3, 6, 7 for group 1) from raw entries
+// prefetched into registers a tile ahead.  The V buffer is single; the chunks of tile t+1 are written
+// as soon as PV(t) has finished the M-tile reading them, so dequantisation and the QK of tile t+1
+// overlap the end of PV(t).  Softmax rescales lazily: O^T and L^T are rescaled in TMEM only when a
+// head's running maximum grows by more than 2^8; the new maxima come from one warp max-reduction per
+// head (redux.sync on order-preserving integer keys).
 #include "attention_common.cuh"
 #include "pipeline.cuh"
 #include "tcgen05.cuh"
@@ -63,11 +66,10 @@ struct TcMisc {
     uint64_t v_free[kTcChunks / 2];
     uint32_t tmem_base;
     int abort_flag;
-    float vmeta[2][kTcRows];    // per entry: -1 masked, else its value scale (1 for FP4, window scale)
+    float vmeta[2][kTcRows];    // per entry: 1 valid, -1 masked
     float zscale[kTcHeads];     // tau * 2^-k_h * log2(e)
     float m[kTcHeads];          // running max, log2 domain
     float alpha[kTcHeads];
-    float lcorr[kTcHeads];      // sum over window rows of p * (1 - scale): their P carries the scale
     float red[4][kTcHeads];
 };
 
@@ -93,29 +95,30 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi)
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
-// Softmax warpgroup barriers (named barrier 1, the 128 threads of warps 0-3).  Every thread of the
-// group executes each of them once per tile, also after a failed wait, so none can be left waiting.
-__device__ __forceinline__ bool group_and(bool v)
+// Warpgroup barriers (named barrier `id`, the 128 threads of one group: 1 for warps 0-3, 2 for warps
+// 4-7).  Every thread of the group executes each of them once per tile, also after a failed wait, so
+// none can be left waiting.
+__device__ __forceinline__ bool group_and(int id, bool v)
 {
     int r;
-    asm volatile("{\n.reg .pred p, q;\nsetp.ne.b32 q, %1, 0;\nbar.red.and.pred p, 1, 128, q;\nselp.b32 %0, 1, 0, p;\n}"
+    asm volatile("{\n.reg .pred p, q;\nsetp.ne.b32 q, %2, 0;\nbar.red.and.pred p, %1, 128, q;\nselp.b32 %0, 1, 0, p;\n}"
                  : "=r"(r)
-                 : "r"((int)v)
+                 : "r"(id), "r"((int)v)
                  : "memory");
     return r != 0;
 }
 
-__device__ __forceinline__ bool group_or(bool v)
+__device__ __forceinline__ bool group_or(int id, bool v)
 {
     int r;
-    asm volatile("{\n.reg .pred p, q;\nsetp.ne.b32 q, %1, 0;\nbar.red.or.pred p, 1, 128, q;\nselp.b32 %0, 1, 0, p;\n}"
+    asm volatile("{\n.reg .pred p, q;\nsetp.ne.b32 q, %2, 0;\nbar.red.or.pred p, %1, 128, q;\nselp.b32 %0, 1, 0, p;\n}"
                  : "=r"(r)
-                 : "r"((int)v)
+                 : "r"(id), "r"((int)v)
                  : "memory");
     return r != 0;
 }
 
-__device__ __forceinline__ void group_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void group_sync(int id) { asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory"); }
 
 // One thread's share of a tile's dequantisation: entry e (tile row) and the four 64-channel chunks of
 // its thread group (group 0: chunks 0, 1, 4, 5; group 1: chunks 2, 3, 6, 7), raw bytes prefetched
@@ -169,8 +172,9 @@ struct TileRows {
                 out[2 * gg + 1] = make_uint4(v[4], v[5], v[6], v[7]);
             }
         } else {
-            // window entry: 64 E4M3 values, exact in fp16; its scale is applied in the softmax
+            // window entry: 64 E4M3 values times the entry's binary32 scale, rounded to fp16
             const uint4 *src = reinterpret_cast<const uint4 *>(r.p + 64 * c);
+            const float fs = r.fscale;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const uint4 w = src[q];
@@ -178,8 +182,10 @@ struct TileRows {
                 uint32_t v[8];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    v[2 * k] = e4m3x2_to_f16x2((uint16_t)(ww[k] & 0xFFFF));
-                    v[2 * k + 1] = e4m3x2_to_f16x2((uint16_t)(ww[k] >> 16));
+                    const uint32_t lo = e4m3x2_to_f16x2((uint16_t)(ww[k] & 0xFFFF));
+                    const uint32_t hi = e4m3x2_to_f16x2((uint16_t)(ww[k] >> 16));
+                    v[2 * k] = pack_f16x2(h_lo(lo) * fs, h_hi(lo) * fs);
+                    v[2 * k + 1] = pack_f16x2(h_lo(hi) * fs, h_hi(hi) * fs);
                 }
                 out[2 * q] = make_uint4(v[0], v[1], v[2], v[3]);
                 out[2 * q + 1] = make_uint4(v[4], v[5], v[6], v[7]);
@@ -269,7 +275,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_split_tc_kernel(AttnArgs a
 
     if (threadIdx.x == 0) {
         mbar_init(&ms.s_full, 1);
-        mbar_init(&ms.p_full, 128);
+        mbar_init(&ms.p_full, 256);   // both groups' halves of P
         mbar_init(&ms.q_ready, 256);
         mbar_init(&ms.o_done, 1);
         mbar_init(&ms.final_bar, 1);
@@ -278,10 +284,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_split_tc_kernel(AttnArgs a
         ms.abort_flag = 0;
         fence_mbar_init();
     }
-    if (threadIdx.x < kTcHeads) {
-        ms.m[threadIdx.x] = -INFINITY;
-        ms.lcorr[threadIdx.x] = 0.f;
-    }
+    if (threadIdx.x < kTcHeads) ms.m[threadIdx.x] = -INFINITY;
     if (threadIdx.x < 32) reinterpret_cast<uint32_t *>(ONES)[threadIdx.x] = 0x3C003C00u;   // fp16 1.0 pairs
     if (warp == 8 && ntiles > 0) {
         tc_alloc(smem_addr(&ms.tmem_base), kTmemCols);
@@ -351,164 +354,116 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_split_tc_kernel(AttnArgs a
             mbar_wait(&ms.final_bar, 0, &no_abort, a.ws, 4);
         }
         __syncwarp();
-    } else if (warp >= 4) {
-        // ------------------------- group 0: Q load, tile metadata, chunks 0, 1, 4, 5 -------------------
-        const int i = threadIdx.x - 128;   // 0..127
-        TileRows rows;
-        rows.load(a, sv, u_begin, u_end, 0, i, 0);
-        load_q(a, ms, Q, b, h0, threadIdx.x);
-        bool ok = true;
-        for (int t = 0; ok && t < ntiles; ++t) {
-            if (t > 0) rows.load(a, sv, u_begin, u_end, t, i, 0);
-            ms.vmeta[t & 1][i] = rows.valid ? (rows.r.swa ? rows.r.fscale : 1.f) : -1.f;
-            ok = dequant_group(ms, V, rows, a, t, i, 0);
-        }
     } else {
-        // ------------------------- group 1: softmax, chunks 2, 3, 6, 7, epilogue ----------------------
-        const int e = threadIdx.x;          // TMEM lane = tile row (entry); channel in the epilogue
-        const int wq = warp;
+        // --------------- softmax groups: group 1 = warps 0-3 (heads 0-31, chunks 2, 3, 6, 7), ---------
+        // --------------- group 0 = warps 4-7 (heads 32-63, chunks 0, 1, 4, 5, tile metadata) ---------
+        const int grp = warp >= 4 ? 0 : 1;
+        const int hh = 1 - grp;              // this group's half of the heads
+        const int bar_id = 2 - grp;          // named barrier of the group
+        const int e = threadIdx.x & 127;     // TMEM lane = tile row (entry); channel in the epilogue
+        const int wq = warp & 3;
         const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
         TileRows rows;
-        rows.load(a, sv, u_begin, u_end, 0, e, 1);
+        rows.load(a, sv, u_begin, u_end, 0, e, grp);
         load_q(a, ms, Q, b, h0, threadIdx.x);
-        bool ok = dequant_group(ms, V, rows, a, 0, e, 1);
-        // the per-head score scales (written by group 0 before q_ready)
-        ok = warp_wait(&ms.q_ready, 0, &ms.abort_flag, a.ws, 1) && ok;
-        ok = group_and(ok);
+        if (grp == 0) ms.vmeta[0][e] = rows.valid ? 1.f : -1.f;
+        bool ok = dequant_group(ms, V, rows, a, 0, e, grp);
+        ok = warp_wait(&ms.q_ready, 0, &ms.abort_flag, a.ws, 1) && ok;   // every head's score scale
+        ok = group_and(bar_id, ok);
         for (int t = 0; ok && t < ntiles; ++t) {
             const uint32_t ph = t & 1;
             bool tok = warp_wait(&ms.s_full, ph, &ms.abort_flag, a.ws, 6) &&
                        warp_wait(&ms.v_ready[0], ph, &ms.abort_flag, a.ws, 7);
-            if (!(ok = group_and(tok))) break;
+            if (!(ok = group_and(bar_id, tok))) break;
             tc_fence_after();
-            const float em = ms.vmeta[ph][e];
-            const bool valid = em >= 0.f;
-            // scores of heads 32*half .. 32*half+31, scaled to the log2 domain (masked rows: -inf)
-            auto load_z = [&](int half, float *zt) {
-                tc_ld32(tl + kColS + 32 * half, zt);
-                tc_wait_ld();
+            const bool valid = ms.vmeta[ph][e] >= 0.f;
+            // scores of this group's 32 heads, in the log2 domain (masked rows: -inf)
+            float zt[32];
+            tc_ld32_sync(tl + kColS + 32 * hh, zt);
 #pragma unroll
-                for (int q = 0; q < 32; ++q) zt[q] = valid ? zt[q] * (em * ms.zscale[32 * half + q]) : -INFINITY;
-            };
+            for (int q = 0; q < 32; ++q) zt[q] = valid ? zt[q] * ms.zscale[32 * hh + q] : -INFINITY;
             bool need = false;
-#pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
-                float zt[32];
-                load_z(half, zt);
 #pragma unroll
-                for (int q = 0; q < 32; ++q) need |= zt[q] > ms.m[32 * half + q] + kLazy;
-            }
-            if (group_or(need)) {
-#pragma unroll 1
-                for (int half = 0; half < 2; ++half) {
-                    float zt[32];
-                    load_z(half, zt);
+            for (int q = 0; q < 32; ++q) need |= zt[q] > ms.m[32 * hh + q] + kLazy;
+            if (group_or(bar_id, need)) {
+                // new maxima: per head one warp max-reduction on order keys, then over the four warps
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) {
-                        float v = zt[q];
-#pragma unroll
-                        for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-                        if (lane == 0) ms.red[wq][32 * half + q] = v;
-                    }
+                for (int q = 0; q < 32; ++q) {
+                    const uint32_t u = __reduce_max_sync(0xffffffffu, order_key(zt[q]));
+                    if (lane == 0) ms.red[wq][32 * hh + q] = key_to_float(u);
                 }
-                group_sync();
-                if (e < kTcHeads) {
-                    const float mt = fmaxf(fmaxf(ms.red[0][e], ms.red[1][e]), fmaxf(ms.red[2][e], ms.red[3][e]));
-                    const float mo = ms.m[e];
+                group_sync(bar_id);
+                if (e < 32) {
+                    const int h = 32 * hh + e;
+                    const float mt = fmaxf(fmaxf(ms.red[0][h], ms.red[1][h]), fmaxf(ms.red[2][h], ms.red[3][h]));
+                    const float mo = ms.m[h];
                     const float mn = fmaxf(mo, mt);
-                    const float al = (mo == -INFINITY) ? 0.f : exp2f(mo - mn);
-                    ms.alpha[e] = al;
-                    ms.m[e] = mn;
-                    ms.lcorr[e] *= al;
+                    ms.alpha[h] = (mo == -INFINITY) ? 0.f : exp2f(mo - mn);
+                    ms.m[h] = mn;
                 }
-                group_sync();
+                group_sync(bar_id);
                 if (t > 0) {
-                    // O^T (4 M-tiles) and L^T columns, per-head factors
+                    // this group's head columns of O^T (4 M-tiles) and of L^T
 #pragma unroll 1
-                    for (int m = 0; m < 10; ++m) {
+                    for (int m = 0; m < 5; ++m) {
                         float o[32];
-                        const uint32_t col = kColO + 32 * m;
-                        tc_ld32(tl + col, o);
-                        tc_wait_ld();
+                        const uint32_t col = (m < 4 ? kColO + 64 * m : kColL) + 32 * hh;
+                        tc_ld32_sync(tl + col, o);
 #pragma unroll
-                        for (int q = 0; q < 32; ++q) o[q] *= ms.alpha[32 * (m & 1) + q];
+                        for (int q = 0; q < 32; ++q) o[q] *= ms.alpha[32 * hh + q];
                         tc_st32(tl + col, o);
                     }
                     tc_wait_st();
                 }
             }
-            const float pv_scale = valid ? em : 0.f;
-            const bool scaled_row = valid && em != 1.f;   // a window entry
-            const bool warp_scaled = __any_sync(0xffffffffu, scaled_row);
-            const float cf = scaled_row ? 1.f - em : 0.f;
-#pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
-                float zt[32];
-                load_z(half, zt);
-                uint32_t pk[16];
+            uint32_t pk[16];
 #pragma unroll
-                for (int q = 0; q < 32; q += 2) {
-                    const float p0 = exp2f(zt[q] - ms.m[32 * half + q] + kPOffset);
-                    const float p1 = exp2f(zt[q + 1] - ms.m[32 * half + q + 1] + kPOffset);
-                    pk[q / 2] = pack_f16x2(p0 * pv_scale, p1 * pv_scale);
-                    zt[q] = p0 * cf;          // reused: the window-row correction of the sums
-                    zt[q + 1] = p1 * cf;
-                }
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj)
-                    *reinterpret_cast<uint4 *>(P + swz((uint32_t)e, (uint32_t)(4 * half + jj))) =
-                        make_uint4(pk[4 * jj], pk[4 * jj + 1], pk[4 * jj + 2], pk[4 * jj + 3]);
-                if (warp_scaled) {
-#pragma unroll
-                    for (int q = 0; q < 32; ++q) {
-                        float v = zt[q];
-#pragma unroll
-                        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                        if (lane == 0) atomicAdd(&ms.lcorr[32 * half + q], v);
-                    }
-                }
+            for (int q = 0; q < 32; q += 2) {
+                const float p0 = exp2f(zt[q] - ms.m[32 * hh + q] + kPOffset);
+                const float p1 = exp2f(zt[q + 1] - ms.m[32 * hh + q + 1] + kPOffset);
+                pk[q / 2] = pack_f16x2(p0, p1);
             }
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj)
+                *reinterpret_cast<uint4 *>(P + swz((uint32_t)e, (uint32_t)(4 * hh + jj))) =
+                    make_uint4(pk[4 * jj], pk[4 * jj + 1], pk[4 * jj + 2], pk[4 * jj + 3]);
             fence_async_smem();
             tc_fence_before();
             mbar_arrive(&ms.p_full);
             // this group's chunks of the next tile, as PV(t) releases them
             if (t + 1 < ntiles) {
-                rows.load(a, sv, u_begin, u_end, t + 1, e, 1);
-                dequant_group(ms, V, rows, a, t + 1, e, 1);
+                rows.load(a, sv, u_begin, u_end, t + 1, e, grp);
+                if (grp == 0) ms.vmeta[(t + 1) & 1][e] = rows.valid ? 1.f : -1.f;
+                dequant_group(ms, V, rows, a, t + 1, e, grp);
             }
         }
-        // ---- epilogue: partial (o, m, l) of this split
+        // ---- epilogue: this group's heads of the split's partial (o, m, l)
         float *po = a.part_o + (((size_t)b * a.splits + s) * a.H + h0) * kLatent;
         float2 *pml = reinterpret_cast<float2 *>(a.part_ml) + ((size_t)b * a.splits + s) * a.H + h0;
         bool eok = ok && warp_wait(&ms.o_done, 0, &ms.abort_flag, a.ws, 8);
-        eok = group_and(eok);
+        eok = group_and(bar_id, eok);
         if (eok) {
             tc_fence_after();
             for (int m = 0; m < 4; ++m) {
+                float o[32];
+                tc_ld32_sync(tl + kColO + 64 * m + 32 * hh, o);
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float o[32];
-                    tc_ld32(tl + kColO + 64 * m + 32 * half, o);
-                    tc_wait_ld();
-#pragma unroll
-                    for (int q = 0; q < 32; ++q) po[(size_t)(32 * half + q) * kLatent + 128 * m + e] = o[q];
-                }
+                for (int q = 0; q < 32; ++q) po[(size_t)(32 * hh + q) * kLatent + 128 * m + e] = o[q];
             }
-            if (warp == 0) {
+            if (wq == 0) {
                 // every row of L^T holds the sums; lane 0's row is shared through shared memory
                 float l[32];
+                tc_ld32_sync(tl + kColL + 32 * hh, l);
+                if (lane == 0) {
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    tc_ld32(tl + kColL + 32 * half, l);
-                    tc_wait_ld();
-                    if (lane == 0) {
-#pragma unroll
-                        for (int q = 0; q < 32; ++q) ms.red[0][32 * half + q] = l[q];
-                    }
+                    for (int q = 0; q < 32; ++q) ms.red[0][32 * hh + q] = l[q];
                 }
             }
-            group_sync();
-            if (e < kTcHeads) pml[e] = make_float2((ms.m[e] - kPOffset) * kLn2, ms.red[0][e] + ms.lcorr[e]);
+            group_sync(bar_id);
+            if (e < 32) {
+                const int h = 32 * hh + e;
+                pml[h] = make_float2((ms.m[h] - kPOffset) * kLn2, ms.red[0][h]);
+            }
         }
     }
     tc_fence_before();

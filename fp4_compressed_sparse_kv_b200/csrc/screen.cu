@@ -519,11 +519,6 @@ struct SeqWords {
 };
 static_assert(sizeof(SeqWords) == kTopkWords * 4, "SeqWords fills one sequence's select words");
 
-__device__ __forceinline__ float key_to_float(uint32_t u)
-{
-    return __uint_as_float((u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u);
-}
-
 // Over a kHistBins-bin histogram h: the bin holding the rank-th largest element (1-based) and that
 // element's rank inside the bin; every thread gets both.  If the counts fall short of rank: bin 0
 // (a threshold that keeps everything).
