@@ -178,7 +178,7 @@ static cudaError_t launch_cc(const AttnArgs &a, cudaStream_t st)
 {
     const size_t smem = (size_t)(HG * kCcRow + kCcTile * kCcRow + kCcTile * HG + 3 * HG) * 4;
     cudaError_t e =
-        cudaFuncSetAttribute(attn_split_cc_kernel<HG>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        allow_dynamic_smem(reinterpret_cast<const void *>(attn_split_cc_kernel<HG>), smem);
     if (e != cudaSuccess) return e;
     const int groups = a.H / HG;
     dim3 grid(a.splits, a.B * groups);

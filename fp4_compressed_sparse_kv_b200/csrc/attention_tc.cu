@@ -479,8 +479,7 @@ int attn_units_per_tile(int H) { return attn_tc_supported(H) ? kTcUnits : 4; }
 cudaError_t launch_attn_tc(const AttnArgs &a, cudaStream_t st)
 {
     static_assert(kTcSmem <= 232448, "shared memory budget");
-    cudaError_t e = cudaFuncSetAttribute(attn_split_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kTcSmem);
+    cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void *>(attn_split_tc_kernel), kTcSmem);
     if (e != cudaSuccess) return e;
     const int groups = a.H / kTcHeads;
     dim3 grid(a.splits, a.B * groups);

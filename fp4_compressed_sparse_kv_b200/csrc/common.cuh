@@ -5,6 +5,8 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/csa.h"
 
 namespace csa {
@@ -68,7 +70,7 @@ inline int attn_splits(int B, int cap, int units_per_tile)
     return s;
 }
 
-constexpr int kTopkWords = 4;
+constexpr int kTopkWords = 8;
 constexpr size_t kQtBytes = 32 * CSA_INDEX_DIM;   // 3 E4M3 terms x 8 heads + 8 zero rows, 128 B each
 constexpr size_t kQmBytes = 64;
 constexpr int kHistBins = 4096;                   // top 12 bits of a 32-bit order key
@@ -113,6 +115,32 @@ inline WsLayout ws_layout(int B, int H, int max_seq_len, int cap, int units_per_
     o = align_up(o + (size_t)B * w.splits * H * 8, 256);
     w.total = o;
     return w;
+}
+
+// Allow `bytes` of dynamic shared memory for kernel `fn` on the current device, calling the runtime
+// only the first time a kernel needs more than it was last allowed there (the setting persists).
+inline cudaError_t allow_dynamic_smem(const void *fn, size_t bytes)
+{
+    struct Entry {
+        const void *fn;
+        int dev;
+        size_t bytes;
+    };
+    static std::mutex mu;
+    static Entry tab[256];
+    static int n = 0;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    int i = 0;
+    while (i < n && !(tab[i].fn == fn && tab[i].dev == dev)) ++i;
+    if (i < n && tab[i].bytes >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e != cudaSuccess) return e;
+    if (i == n && n < 256) tab[n++] = Entry{fn, dev, bytes};
+    else if (i < n) tab[i].bytes = bytes;
+    return cudaSuccess;
 }
 
 // ------------------------------------------------------------------------------------------------

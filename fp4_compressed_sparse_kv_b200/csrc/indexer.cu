@@ -441,7 +441,7 @@ static int num_sms()
 cudaError_t launch_block_scores(const ScoreArgs &args, cudaStream_t st)
 {
     const size_t smem = sizeof(ScoreSmem);
-    cudaError_t e = cudaFuncSetAttribute(block_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void *>(block_score_kernel), smem);
     if (e != cudaSuccess) return e;
     const long long total = (long long)args.B * args.items_per_seq;
     if (total == 0) return cudaSuccess;
@@ -505,7 +505,7 @@ cudaError_t launch_block_scores_list(const uint8_t *keys, int num_pages, const c
     a.score_stride = score_stride;
     a.ws = ws;
     const size_t smem = sizeof(ScoreSmem);
-    cudaError_t e = cudaFuncSetAttribute(block_score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void *>(block_score_kernel), smem);
     if (e != cudaSuccess) return e;
     block_score_kernel<<<num_sms(), kScoreThreads, smem, st>>>(a);
     return cudaGetLastError();
@@ -517,7 +517,7 @@ cudaError_t launch_topk(const float *scores, int score_stride, const int32_t *se
 {
     const size_t smem =
         (size_t)kTopkHistWords * 4 + (size_t)(max_candidates < kTopkCacheKeys ? max_candidates : kTopkCacheKeys) * 4;
-    cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void *>(topk_kernel), smem);
     if (e != cudaSuccess) return e;
     topk_kernel<<<B, kTopkThreads, smem, st>>>(scores, score_stride, seq_len, max_seq_len, pool, pool_count, pool_cap,
                                                k, out_blocks, out_count, ws);

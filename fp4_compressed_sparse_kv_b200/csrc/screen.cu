@@ -513,9 +513,10 @@ __global__ void __launch_bounds__(kScrThreads, 1) screen_kernel(const __grid_con
 constexpr int kClsThreads = 256;
 constexpr uint8_t kOut = 0, kSure = 1, kUncertain = 2, kChosen = 3, kTie = 4;
 
-// Per-sequence words: [0] sure blocks, [1] uncertain blocks, [2] order key of the widest interval.
+// Per-sequence words: sure blocks, uncertain blocks, order key of the widest interval, and the
+// first-level histogram bin of the k-th largest lower bound with that element's rank inside it.
 struct SeqWords {
-    uint32_t n_sure, n_uncertain, wmax_key, pad;
+    uint32_t n_sure, n_uncertain, wmax_key, bin1, r1, pad[3];
 };
 static_assert(sizeof(SeqWords) == kTopkWords * 4, "SeqWords fills one sequence's select words");
 
@@ -609,6 +610,10 @@ __global__ void __launch_bounds__(kClsThreads) classify_a_kernel(const ClsArgs a
     int bin1;
     uint32_t r1;
     rank_bin<kClsThreads>(a.hist + (size_t)b * kHistBins, (uint32_t)a.k, scratch, &bin1, &r1);
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        a.words[b].bin1 = (uint32_t)bin1;
+        a.words[b].r1 = r1;
+    }
     const float *lp = a.lo + (size_t)b * a.stride;
     const float *hp = a.hi + (size_t)b * a.stride;
     uint32_t *h2 = a.hist2 + (size_t)b * kHistBins;
@@ -630,10 +635,10 @@ __global__ void __launch_bounds__(kClsThreads) classify_b_kernel(const ClsArgs a
     const int b = blockIdx.y, lane = threadIdx.x & 31;
     int n, i0, i1;
     if (!cls_chunk(a, b, n, i0, i1)) return;
-    int bin1, bin2;
-    uint32_t r1, r2;
-    rank_bin<kClsThreads>(a.hist + (size_t)b * kHistBins, (uint32_t)a.k, scratch, &bin1, &r1);
-    rank_bin<kClsThreads>(a.hist2 + (size_t)b * kHistBins, r1, scratch, &bin2, &r2);
+    const int bin1 = (int)a.words[b].bin1;
+    int bin2;
+    uint32_t r2;
+    rank_bin<kClsThreads>(a.hist2 + (size_t)b * kHistBins, a.words[b].r1, scratch, &bin2, &r2);
     const uint32_t T = ((uint32_t)bin1 << 20) | ((uint32_t)bin2 << 8);
     const uint32_t wkey = a.words[b].wmax_key;
     const float wmax = key_to_float(wkey);
@@ -863,6 +868,45 @@ cudaError_t tensor_map_encoder(PFN_cuTensorMapEncodeTiled_v12000 *out)
     return cudaSuccess;
 }
 
+// The keys' tensor map, re-encoded only when the key pool changes (the last one per device is kept).
+cudaError_t keys_tensor_map(const uint8_t *keys, int num_pages, CUtensorMap *out)
+{
+    struct Cached {
+        const uint8_t *keys;
+        int num_pages;
+        CUtensorMap map;
+    };
+    static std::mutex mu;
+    static Cached cache[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) {
+        std::lock_guard<std::mutex> lock(mu);
+        if (cache[dev].keys == keys && cache[dev].num_pages == num_pages) {
+            *out = cache[dev].map;
+            return cudaSuccess;
+        }
+    }
+    PFN_cuTensorMapEncodeTiled_v12000 encode;
+    if ((e = tensor_map_encoder(&encode)) != cudaSuccess) return e;
+    const cuuint64_t dims[2] = {(cuuint64_t)kIdxDim, (cuuint64_t)num_pages * kPage};
+    const cuuint64_t strides[1] = {(cuuint64_t)kIdxDim};
+    const cuuint32_t box[2] = {(cuuint32_t)kIdxDim, (cuuint32_t)kPage};
+    const cuuint32_t estr[2] = {1, 1};
+    if (encode(out, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(keys), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    if (dev >= 0 && dev < 64) {
+        std::lock_guard<std::mutex> lock(mu);
+        cache[dev].keys = keys;
+        cache[dev].num_pages = num_pages;
+        cache[dev].map = *out;
+    }
+    return cudaSuccess;
+}
+
 int g_sm_count[64];
 
 int sm_count()
@@ -888,17 +932,8 @@ cudaError_t launch_screen_bounds(const uint8_t *keys, int num_pages, const csa_b
                                  cudaStream_t st)
 {
     cudaError_t e;
-    PFN_cuTensorMapEncodeTiled_v12000 encode;
-    if ((e = tensor_map_encoder(&encode)) != cudaSuccess) return e;
     CUtensorMap map;
-    const cuuint64_t dims[2] = {(cuuint64_t)kIdxDim, (cuuint64_t)num_pages * kPage};
-    const cuuint64_t strides[1] = {(cuuint64_t)kIdxDim};
-    const cuuint32_t box[2] = {(cuuint32_t)kIdxDim, (cuuint32_t)kPage};
-    const cuuint32_t estr[2] = {1, 1};
-    if (encode(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(keys), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return cudaErrorInvalidValue;
+    if ((e = keys_tensor_map(keys, num_pages, &map)) != cudaSuccess) return e;
 
     qterm_kernel<<<bt.B, 256, 0, st>>>(iq, iw, qt, reinterpret_cast<QMeta *>(qm), list_count, hist, hist2,
                                        reinterpret_cast<uint32_t *>(words));
@@ -924,7 +959,7 @@ cudaError_t launch_screen_bounds(const uint8_t *keys, int num_pages, const csa_b
     sa.hist = hist;
     sa.ws = ws;
     const size_t smem = sizeof(ScrSmem) + 1024;
-    if ((e = cudaFuncSetAttribute(screen_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+    if ((e = allow_dynamic_smem(reinterpret_cast<const void *>(screen_kernel), smem)) != cudaSuccess)
         return e;
     screen_kernel<<<grid, kScrThreads, smem, st>>>(map, sa);
     return cudaGetLastError();
@@ -970,7 +1005,7 @@ cudaError_t launch_finalize(const float *scores, int score_stride, const csa_bat
 {
     const size_t smem = ((size_t)kFinWarps * 256 + kFinCache) * 4 + kFinStatusCache;
     static_assert(2 * kFinRankMax <= kFinCache, "rank-path keys and ids share the key cache");
-    cudaError_t e = cudaFuncSetAttribute(finalize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void *>(finalize_kernel), smem);
     if (e != cudaSuccess) return e;
     finalize_kernel<<<bt.B, kFinThreads, smem, st>>>(scores, score_stride, bt.seq_len, bt.max_seq_len, status, sstride,
                                                       uslice, reinterpret_cast<const SeqWords *>(words), stride, k,
