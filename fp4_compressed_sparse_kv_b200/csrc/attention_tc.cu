@@ -126,8 +126,19 @@ __device__ __forceinline__ void group_sync(int id) { asm volatile("bar.sync %0, 
 struct TileRows {
     EntryRef r;
     bool valid;
-    uint4 code[8];     // code bytes of the group's chunks: 64 B at 64*g, 64 B at 128 + 64*g
+    uint4 code[8];     // FP4 entry: code bytes of the group's chunks (64 B at 64*g, 64 B at 128 + 64*g);
+                       // window entry: the 128 values of the chunk pair being written
     uint2 scl[2];      // their scale words
+
+    // Window entry: start loading the values of chunk pair `pair` (chunks 2g + 4 pair and the next).
+    __device__ __forceinline__ void fetch_window_pair(int pair, int g)
+    {
+        if (valid && r.swa) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(r.p + 64 * (2 * g + 4 * pair));
+#pragma unroll
+            for (int q = 0; q < 8; ++q) code[q] = src[q];
+        }
+    }
 
     __device__ __forceinline__ void load(const AttnArgs &a, const SeqView &sv, int u_begin, int u_end, int t, int e,
                                          int g)
@@ -172,12 +183,12 @@ struct TileRows {
                 out[2 * gg + 1] = make_uint4(v[4], v[5], v[6], v[7]);
             }
         } else {
-            // window entry: 64 E4M3 values times the entry's binary32 scale, rounded to fp16
-            const uint4 *src = reinterpret_cast<const uint4 *>(r.p + 64 * c);
+            // window entry: 64 E4M3 values (fetched with its chunk pair) times the entry's binary32
+            // scale, rounded to fp16
             const float fs = r.fscale;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                const uint4 w = src[q];
+                const uint4 w = code[4 * (cs & 1) + q];
                 const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
                 uint32_t v[8];
 #pragma unroll
@@ -197,14 +208,17 @@ struct TileRows {
 };
 
 // Dequantise this group's four chunks of tile t into V (waiting for PV(t-1) to release each pair).
-__device__ __forceinline__ bool dequant_group(TcMisc &ms, uint8_t *V, const TileRows &rows, const AttnArgs &a, int t,
-                                              int e, int g)
+__device__ __forceinline__ bool dequant_group(TcMisc &ms, uint8_t *V, TileRows &rows, const AttnArgs &a, int t, int e,
+                                              int g)
 {
     bool ok = true;
 #pragma unroll
     for (int cs = 0; cs < 4; ++cs) {
         const int c = 2 * g + (cs & 1) + 4 * (cs >> 1);
-        if (t > 0 && (cs & 1) == 0) ok = ok && warp_wait(&ms.v_free[c >> 1], (t - 1) & 1, &ms.abort_flag, a.ws, 5);
+        if ((cs & 1) == 0) {
+            rows.fetch_window_pair(cs >> 1, g);   // in flight while PV(t-1) releases the pair
+            if (t > 0) ok = ok && warp_wait(&ms.v_free[c >> 1], (t - 1) & 1, &ms.abort_flag, a.ws, 5);
+        }
         if (ok) rows.write(V, e, c, cs);
         fence_async_smem();
         mbar_arrive(&ms.v_ready[c]);
