@@ -278,6 +278,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_split_tc_kernel(AttnArgs a
     TcMisc &ms = *reinterpret_cast<TcMisc *>(base + kOffMisc);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    grid_dep_wait();   // the selected blocks of the previous grid
     const int s = blockIdx.x, b = blockIdx.y / head_groups, hg = blockIdx.y % head_groups;
     const int h0 = hg * kTcHeads;
 
@@ -497,8 +498,7 @@ cudaError_t launch_attn_tc(const AttnArgs &a, cudaStream_t st)
     if (e != cudaSuccess) return e;
     const int groups = a.H / kTcHeads;
     dim3 grid(a.splits, a.B * groups);
-    attn_split_tc_kernel<<<grid, kTcThreads, kTcSmem, st>>>(a, groups);
-    return cudaGetLastError();
+    return launch_overlapped(attn_split_tc_kernel, grid, dim3(kTcThreads), kTcSmem, st, a, groups);
 }
 
 }  // namespace csa

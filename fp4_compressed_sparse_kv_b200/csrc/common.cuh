@@ -143,6 +143,26 @@ inline cudaError_t allow_dynamic_smem(const void *fn, size_t bytes)
     return cudaSuccess;
 }
 
+// Launch `kernel` so that it may start before the previous grid of the stream completes: the
+// previous grid lets it be scheduled (grid_dep_launch) and the kernel waits for the previous grid's
+// results where it needs them (grid_dep_wait).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_overlapped(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                     Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
+}
+
 // ------------------------------------------------------------------------------------------------
 // Device status word: the first error wins; its detail is the offending index.
 // ------------------------------------------------------------------------------------------------

@@ -95,6 +95,13 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
     return r != 0;
 }
 
+// Programmatic dependent launch.  grid_dep_wait: wait until the previous grid of the stream has
+// completed and its memory is visible (call before touching anything it writes); grid_dep_launch:
+// allow the next grid of the stream to be scheduled.  Both do nothing for grids launched without the
+// programmatic-serialization attribute.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Order this thread's generic-proxy shared-memory accesses with later async-proxy accesses (bulk
 // copies, tensor-core operand reads) of the same memory.
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }

@@ -93,6 +93,7 @@ __global__ void __launch_bounds__(256) qterm_kernel(const uint16_t *__restrict__
                                                     uint32_t *__restrict__ hist2, uint32_t *__restrict__ seq_words)
 {
     const int b = blockIdx.x, h = threadIdx.x >> 5, l = threadIdx.x & 31;
+    grid_dep_launch();   // the screen may start streaming keys meanwhile
     // the counters the later steps accumulate into start from zero on every call
     if (b == 0 && threadIdx.x == 0 && list_count) *list_count = 0;
     for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) {
@@ -343,6 +344,7 @@ __global__ void __launch_bounds__(kScrThreads, 1) screen_kernel(const __grid_con
             sm.ring[k % kScrRing] = it;
         };
         long long issued = 0;
+        bool q_visible = false;   // the query terms of the previous grid have been waited for
         for (long long k = 0; k < n_items; ++k) {
             if ((k & 31) == 0) {
                 resolve32(k);
@@ -361,6 +363,10 @@ __global__ void __launch_bounds__(kScrThreads, 1) screen_kernel(const __grid_con
                         tma_load_2d(sm.keys[st], &tmap, 0, it.p0 * kPage, &sm.full[st]);
                         if (it.p1 >= 0) tma_load_2d(sm.keys[st] + kScrPageBytes, &tmap, 0, it.p1 * kPage, &sm.full[st]);
                         if (need_q) {
+                            if (!q_visible) {
+                                grid_dep_wait();
+                                q_visible = true;
+                            }
                             bulk_g2s(sm.qt[st], a.qt + (size_t)it.b * kScrQtBytes, kScrQtBytes, &sm.full[st]);
                             sm.stage_b[st] = it.b;
                         }
@@ -426,6 +432,7 @@ __global__ void __launch_bounds__(kScrThreads, 1) screen_kernel(const __grid_con
     } else {
         // ---------------- epilogue group g: tiles k = g, g + 2, ...; thread = tile row = TMEM lane ----
         const int g = (warp - kScrEpiWarp0) >> 2;
+        grid_dep_wait();   // the screening constants and the zeroed histogram
         const int quad = warp & 3;
         const int r = 32 * quad + lane;
         const uint32_t tl = tmem + ((uint32_t)(32 * quad) << 16);
@@ -706,6 +713,7 @@ __global__ void __launch_bounds__(kFinThreads, 1) finalize_kernel(
     __shared__ uint32_t scratch[72];
     __shared__ uint32_t sel[2];
     const int b = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    grid_dep_launch();   // the attention may be scheduled meanwhile
     const int L = seq_len[b];
     int32_t *out = out_blocks + (size_t)b * k;
     if (L < 1 || L > max_seq_len) {   // reported by the classification
@@ -961,8 +969,7 @@ cudaError_t launch_screen_bounds(const uint8_t *keys, int num_pages, const csa_b
     const size_t smem = sizeof(ScrSmem) + 1024;
     if ((e = allow_dynamic_smem(reinterpret_cast<const void *>(screen_kernel), smem)) != cudaSuccess)
         return e;
-    screen_kernel<<<grid, kScrThreads, smem, st>>>(map, sa);
-    return cudaGetLastError();
+    return launch_overlapped(screen_kernel, dim3(grid), dim3(kScrThreads), smem, st, map, sa);
 }
 
 cudaError_t launch_classify(const float *lo, const float *hi, int stride, const csa_batch &bt, int k,
