@@ -174,9 +174,9 @@ __global__ void __launch_bounds__(256) qterm_kernel(const uint16_t *__restrict__
 // image.  As soon as a stage lands, warp 1 issues the four K=32 MMAs of its tile into one of six
 // 32-column TMEM accumulators and one of two row-max groups (warps 2-5, 6-9; thread = row) writes
 // each row's largest |key| beside that accumulator; the stage is then free again (the MMA's commit
-// and the 128 row-max threads release it), so nearly all stages stay in flight.  Two groups of four epilogue warps (thread =
-// tile row = TMEM lane) take the tiles in turn (tile k: accumulator k mod 6, group k mod 2) and
-// turn accumulator and row maxima into per-block bounds.
+// and the 128 row-max threads release it), so nearly all stages stay in flight.  Two groups of four
+// epilogue warps (thread = tile row = TMEM lane) take the tiles in turn (tile k: accumulator k mod 6,
+// group k mod 2) and turn accumulator and row maxima into per-block bounds.
 // ------------------------------------------------------------------------------------------------
 struct ScreenArgs {
     const int32_t *seq_len;
