@@ -82,6 +82,30 @@ def test_bad_host_arguments_return_before_launch(lib):
     assert lib.csa_kv_pack_fp4(null, null, null, null, null, 0, null, 0, null) == 0
 
 
+def test_screen_and_full_indexer_host_checks(lib):
+    """Argument and workspace checks of the screened Full indexer happen on the host, before any
+    launch: null or misaligned pointers, a bounds stride below ceil(max_seq_len / 8), and a workspace
+    smaller than csa_workspace_bytes asks for."""
+    from fp4_compressed_sparse_kv_b200 import csa
+    null = None
+    fake = ctypes.c_void_p(0x1000)
+    lay = csa.KVLayerC(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 64, 1)
+    bat = csa.BatchC(2, 0x1000, 0x1000, 64, 0x1000, 4096)   # B=2, max_seq_len 4,096: 512 blocks
+    args = (ctypes.byref(lay), ctypes.byref(bat), fake, fake, fake, fake)
+    assert lib.csa_indexer_screen_bounds(null, null, null, null, null, null, 512, null, 0, null) == 1
+    assert lib.csa_indexer_screen_bounds(*args, 511, fake, 1 << 30, null) == 1       # stride too small
+    odd = ctypes.c_void_p(0x1004)
+    assert lib.csa_indexer_screen_bounds(ctypes.byref(lay), ctypes.byref(bat), fake, fake, odd, fake, 512, fake,
+                                         1 << 30, null) == 1
+    need = lib.csa_workspace_bytes(2, 16, 4096, 1)
+    assert need > 0
+    assert lib.csa_indexer_screen_bounds(*args, 512, fake, 256, null) == 3            # workspace too small
+    assert lib.csa_indexer_full(ctypes.byref(lay), ctypes.byref(bat), fake, fake, 64, fake, fake, fake, 300,
+                                null) == 3
+    assert lib.csa_indexer_full(ctypes.byref(lay), ctypes.byref(bat), fake, fake, 0, fake, fake, fake, 1 << 30,
+                                null) == 1                                               # k out of range
+
+
 def test_binding_refuses_host_tensors():
     import torch
     from fp4_compressed_sparse_kv_b200 import csa
