@@ -60,6 +60,8 @@ def lib():
             getattr(L, n).argtypes = [i64, P, P]
         L.ora_pack_tokens.restype = None
         L.ora_pack_tokens.argtypes = [i64, P, P, P, P, P, P, P]
+        L.ora_norm_rope.restype = None
+        L.ora_norm_rope.argtypes = [i64, P, P, P, P]
         L.ora_index_score.restype = ctypes.c_float
         L.ora_index_score.argtypes = [P, P, P]
         L.ora_index_scores.restype = None
@@ -136,6 +138,19 @@ def pack_tokens(latent_bf16, key_bf16, with_swa=True):
     lib().ora_pack_tokens(n, _p(lat), _p(key), _p(out["codes"]), _p(out["scales"]),
                           _p(out["key8"]), _p(swa) if with_swa else None,
                           _p(swa_scale) if with_swa else None)
+    return out
+
+
+def norm_rope(latent_bf16, weight, cos_sin):
+    """RMSNorm (weight [512], eps 1e-6) then RoPE on channels 448..511 of n pre-norm latents, in the
+    binary32 order of ora_norm_rope.  latent_bf16 uint16 [n,512]; cos_sin float32 [n,32,2] (cos_i,
+    sin_i of pair i = channels 448+2i, 449+2i).  Returns bf16 bit patterns uint16 [n,512]."""
+    x = _c(latent_bf16, np.uint16).reshape(-1, LATENT)
+    n = x.shape[0]
+    w = _c(weight, np.float32).reshape(LATENT)
+    cs = _c(cos_sin, np.float32).reshape(n, 32, 2)
+    out = np.zeros((n, LATENT), np.uint16)
+    lib().ora_norm_rope(n, _p(x), _p(w), _p(cs), _p(out))
     return out
 
 

@@ -163,6 +163,70 @@ void ora_pack_swa(const uint16_t *latent, uint8_t *swa, float *swa_scale)
         swa[c] = (scale == 0.0f) ? 0 : ora_e4m3_encode(bf16_to_f32(latent[c]) / scale);
 }
 
+/* binary32 -> bf16, round to nearest even (NaN stays a quiet NaN). */
+static uint16_t f32_to_bf16(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7FFFFFFFu) > 0x7F800000u)
+        return (uint16_t)((u >> 16) | 0x40u);
+    u += 0x7FFFu + ((u >> 16) & 1u);
+    return (uint16_t)(u >> 16);
+}
+
+/* ---------------------------------------------------------------------------------------------
+ * Step 0, before the pack: RMSNorm of the 512-channel pre-norm latent with a caller-given weight,
+ * then the rotary embedding of channels 448..511 with caller-given (cos, sin) per pair, rounded to
+ * bf16.  The pages fix only that the latent is RMS-normalised (weights of magnitude about 1) and
+ * rotated by RoPE, which keeps its norm ([ailily] §三); the arithmetic is this build's reading, in
+ * binary32, in exactly this order:
+ *   s_g = FMA chain of v_c * v_c over c = 16g .. 16g+15, from 0 (g = 0..31);
+ *   for d = 16, 8, 4, 2, 1: s_g <- s_g + s_(g xor d) for every g at once; ss = s_0;
+ *   r = 1 / sqrt(ss / 512 + 1e-6), every operation correctly rounded;
+ *   y_c = (v_c * r) * w_c;
+ *   pair i = 0..31, (a, b) = (y_(448+2i), y_(449+2i)):
+ *     y_(448+2i) = (a * cos_i) - (b * sin_i),  y_(449+2i) = (a * sin_i) + (b * cos_i);
+ *   out_c = bf16(y_c).
+ * n tokens: x bf16 [n][512], w [512], cs [n][32][2] = (cos_i, sin_i), out bf16 [n][512].
+ * ------------------------------------------------------------------------------------------- */
+void ora_norm_rope(int64_t n, const uint16_t *x, const float *w, const float *cs, uint16_t *out)
+{
+    for (int64_t t = 0; t < n; ++t) {
+        const uint16_t *xt = x + 512 * t;
+        float v[512], y[512], s[32], s2[32];
+        for (int c = 0; c < 512; ++c)
+            v[c] = bf16_to_f32(xt[c]);
+        for (int g = 0; g < 32; ++g) {
+            float acc = 0.0f;
+            for (int c = 16 * g; c < 16 * g + 16; ++c)
+                acc = fmaf(v[c], v[c], acc);
+            s[g] = acc;
+        }
+        for (int d = 16; d >= 1; d >>= 1) {
+            for (int g = 0; g < 32; ++g)
+                s2[g] = s[g] + s[g ^ d];
+            memcpy(s, s2, sizeof s);
+        }
+        const float mean = s[0] / 512.0f;
+        const float q = sqrtf(mean + 1e-6f);
+        const float r = 1.0f / q;
+        for (int c = 0; c < 512; ++c) {
+            const float vr = v[c] * r;
+            y[c] = vr * w[c];
+        }
+        const float *cst = cs + 64 * t;
+        for (int i = 0; i < 32; ++i) {
+            const float a = y[448 + 2 * i], b = y[449 + 2 * i];
+            const float co = cst[2 * i], si = cst[2 * i + 1];
+            const float ac = a * co, bs = b * si, as = a * si, bc = b * co;
+            y[448 + 2 * i] = ac - bs;
+            y[449 + 2 * i] = as + bc;
+        }
+        for (int c = 0; c < 512; ++c)
+            out[512 * t + c] = f32_to_bf16(y[c]);
+    }
+}
+
 /* n tokens, outputs packed densely per token.  swa/swa_scale may be NULL. */
 void ora_pack_tokens(int64_t n, const uint16_t *latent, const uint16_t *key, uint8_t *codes,
                      uint8_t *scales, uint8_t *key8, uint8_t *swa, float *swa_scale)
