@@ -57,7 +57,7 @@ class LayerStepC(ctypes.Structure):
 EXPORTS = ["csa_workspace_bytes", "csa_workspace_init", "csa_kv_pack_fp4", "csa_indexer_full",
            "csa_indexer_reindex", "csa_indexer_block_scores", "csa_topk_blocks", "csa_index_reuse", "csa_sparse_decode_attn", "csa_decode_layer",
            "csa_check_device_error", "csa_status_string", "csa_indexer_full_noalloc",
-           "csa_indexer_screen_bounds"]
+           "csa_indexer_screen_bounds", "csa_kv_norm_rope_pack_fp4"]
 
 _lib = None
 
@@ -79,6 +79,8 @@ def lib():
     L.csa_workspace_init.argtypes = [P, sz, P]
     L.csa_kv_pack_fp4.restype = st
     L.csa_kv_pack_fp4.argtypes = [ctypes.POINTER(KVLayerC), P, P, P, P, i32, P, sz, P]
+    L.csa_kv_norm_rope_pack_fp4.restype = st
+    L.csa_kv_norm_rope_pack_fp4.argtypes = [ctypes.POINTER(KVLayerC), P, P, P, P, P, P, i32, P, sz, P]
     L.csa_indexer_full.restype = st
     L.csa_indexer_full.argtypes = [ctypes.POINTER(KVLayerC), ctypes.POINTER(BatchC), P, P, i32, P, P,
                                    P, sz, P]
@@ -207,6 +209,19 @@ def kv_pack_fp4(layer, latent, idx_key, slot, swa_slot, ws, stream=None):
                                  _ptr(_bits(idx_key), "idx_key"), _ptr(slot, "slot"),
                                  _ptr(swa_slot, "swa_slot"), n, _ptr(ws, "ws"), ws.numel(),
                                  _stream(stream)), "csa_kv_pack_fp4")
+
+
+def kv_norm_rope_pack_fp4(layer, latent_prenorm, norm_weight, rope_cos_sin, idx_key, slot, swa_slot, ws,
+                          stream=None):
+    """Pack from the pre-norm latent: RMSNorm (norm_weight float32 [512]), RoPE on channels 448..511
+    (rope_cos_sin float32 [n, 32, 2] of (cos, sin) pairs), bf16, then the FP4 / E4M3 / FP8 pack."""
+    n = int(slot.numel())
+    lc = layer.c()
+    _check(lib().csa_kv_norm_rope_pack_fp4(ctypes.byref(lc), _ptr(_bits(latent_prenorm), "latent_prenorm"),
+                                           _ptr(norm_weight, "norm_weight"), _ptr(rope_cos_sin, "rope_cos_sin"),
+                                           _ptr(_bits(idx_key), "idx_key"), _ptr(slot, "slot"),
+                                           _ptr(swa_slot, "swa_slot"), n, _ptr(ws, "ws"), ws.numel(),
+                                           _stream(stream)), "csa_kv_norm_rope_pack_fp4")
 
 
 def indexer_full(layer, batch, iq, iw, k, out_blocks, out_count, ws, stream=None):

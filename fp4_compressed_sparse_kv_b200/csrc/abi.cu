@@ -10,6 +10,9 @@ namespace csa {
 struct ScoreArgs;
 cudaError_t launch_kv_pack(const csa_kv_layer &layer, const uint16_t *latent, const uint16_t *idx_key,
                            const int64_t *slot, const int32_t *swa_slot, int n, void *ws, cudaStream_t st);
+cudaError_t launch_kv_norm_rope_pack(const csa_kv_layer &layer, const uint16_t *latent, const float *norm_w,
+                                     const float *rope_cs, const uint16_t *idx_key, const int64_t *slot,
+                                     const int32_t *swa_slot, int n, void *ws, cudaStream_t st);
 cudaError_t launch_topk(const float *scores, int score_stride, const int32_t *seq_len, int max_seq_len,
                         const int32_t *pool, const int32_t *pool_count, int pool_cap, int k, int B,
                         int32_t *out_blocks, int32_t *out_count, int max_candidates, void *ws, cudaStream_t st);
@@ -105,6 +108,24 @@ csa_status csa_kv_pack_fp4(const csa_kv_layer *layer, const uint16_t *latent, co
     if (!ws || !aligned16(ws)) return CSA_ERR_INVALID_ARG;
     if (ws_bytes < kHeaderBytes) return CSA_ERR_WORKSPACE;
     return cuda_status(launch_kv_pack(*layer, latent, idx_key, slot, swa_slot, n, ws, (cudaStream_t)stream));
+}
+
+csa_status csa_kv_norm_rope_pack_fp4(const csa_kv_layer *layer, const uint16_t *latent_prenorm,
+                                     const float *norm_weight, const float *rope_cos_sin, const uint16_t *idx_key,
+                                     const int64_t *slot, const int32_t *swa_slot, int32_t n, void *ws,
+                                     size_t ws_bytes, void *stream)
+{
+    if (n < 0) return CSA_ERR_INVALID_ARG;
+    if (n == 0) return CSA_OK;
+    if (!layer_ok(layer, swa_slot != nullptr)) return CSA_ERR_INVALID_ARG;
+    if (!latent_prenorm || !norm_weight || !rope_cos_sin || !idx_key || !slot || !aligned16(latent_prenorm) ||
+        !aligned16(norm_weight) || !aligned16(rope_cos_sin) || !aligned16(idx_key) || !aligned16(slot))
+        return CSA_ERR_INVALID_ARG;
+    if (swa_slot && !aligned16(swa_slot)) return CSA_ERR_INVALID_ARG;
+    if (!ws || !aligned16(ws)) return CSA_ERR_INVALID_ARG;
+    if (ws_bytes < kHeaderBytes) return CSA_ERR_WORKSPACE;
+    return cuda_status(launch_kv_norm_rope_pack(*layer, latent_prenorm, norm_weight, rope_cos_sin, idx_key, slot,
+                                                swa_slot, n, ws, (cudaStream_t)stream));
 }
 
 csa_status csa_indexer_block_scores(const csa_kv_layer *layer, const csa_batch *batch, const uint16_t *iq,

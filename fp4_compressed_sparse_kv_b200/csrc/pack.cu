@@ -9,15 +9,27 @@
 // one E4M3 scale: its amax needs no cross-lane step, and its 16 codes are one 8-byte store.  The
 // window entry needs the token's amax, a 5-step warp max.  Loads are 2 x 16 B per lane (latent) and
 // 8 B per lane (key), all coalesced; HBM-bound streaming.
+//
+// The norm variant starts from the pre-norm latent (ailily.cc article, section 三: the KV latent is
+// RMS-normalised, with weights of magnitude about 1, and rotated by RoPE, which keeps its norm): in
+// binary32, lane g forms the FMA chain of its 16 squares, an xor butterfly (16, 8, 4, 2, 1) sums the
+// lanes, r = 1 / sqrt(sum / 512 + 1e-6) with correctly rounded operations, y = (v * r) * weight; lanes
+// 28-31 then rotate their channel pairs (448 + 2i, 449 + 2i) with the caller's (cos_i, sin_i), every
+// product and sum rounded on its own; the result is rounded to bf16 and packed as above.
+#include <cuda_bf16.h>
+
 #include "common.cuh"
 #include "convert.cuh"
 
 namespace csa {
 
+template <bool kNorm>
 __global__ void __launch_bounds__(256) kv_pack_kernel(csa_kv_layer layer, const uint16_t *__restrict__ latent,
                                                       const uint16_t *__restrict__ idx_key,
                                                       const int64_t *__restrict__ slot,
-                                                      const int32_t *__restrict__ swa_slot, int n, void *ws)
+                                                      const int32_t *__restrict__ swa_slot, int n, void *ws,
+                                                      const float *__restrict__ norm_w,
+                                                      const float *__restrict__ rope_cs)
 {
     const int tok = blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
@@ -38,6 +50,40 @@ __global__ void __launch_bounds__(256) kv_pack_kernel(csa_kv_layer layer, const 
     for (int i = 0; i < 8; ++i) {
         x[2 * i] = bf16_lo(w[i]);
         x[2 * i + 1] = bf16_hi(w[i]);
+    }
+    if (kNorm) {
+        float acc = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) acc = __fmaf_rn(x[i], x[i], acc);
+#pragma unroll
+        for (int d = 16; d > 0; d >>= 1) acc = __fadd_rn(acc, __shfl_xor_sync(0xffffffffu, acc, d));
+        const float r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(acc, 512.0f), 1e-6f)));
+        const float4 *wp = reinterpret_cast<const float4 *>(norm_w + 16 * lane);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float4 wv = wp[q];
+            x[4 * q] = __fmul_rn(__fmul_rn(x[4 * q], r), wv.x);
+            x[4 * q + 1] = __fmul_rn(__fmul_rn(x[4 * q + 1], r), wv.y);
+            x[4 * q + 2] = __fmul_rn(__fmul_rn(x[4 * q + 2], r), wv.z);
+            x[4 * q + 3] = __fmul_rn(__fmul_rn(x[4 * q + 3], r), wv.w);
+        }
+        if (lane >= 28) {   // channels 448..511: pairs 8 (lane - 28) .. 8 (lane - 28) + 7
+            const float4 *cp = reinterpret_cast<const float4 *>(rope_cs + (size_t)tok * 64 + 16 * (lane - 28));
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float4 c2 = cp[q];   // (cos, sin) of two pairs
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const float co = h ? c2.z : c2.x, si = h ? c2.w : c2.y;
+                    const int m = 2 * q + h;
+                    const float a = x[2 * m], b = x[2 * m + 1];
+                    x[2 * m] = __fsub_rn(__fmul_rn(a, co), __fmul_rn(b, si));
+                    x[2 * m + 1] = __fadd_rn(__fmul_rn(a, si), __fmul_rn(b, co));
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) x[i] = __bfloat162float(__float2bfloat16_rn(x[i]));
     }
     float amax = 0.f;
 #pragma unroll
@@ -90,7 +136,18 @@ cudaError_t launch_kv_pack(const csa_kv_layer &layer, const uint16_t *latent, co
                            const int64_t *slot, const int32_t *swa_slot, int n, void *ws, cudaStream_t st)
 {
     if (n == 0) return cudaSuccess;
-    kv_pack_kernel<<<(n + 7) / 8, 256, 0, st>>>(layer, latent, idx_key, slot, swa_slot, n, ws);
+    kv_pack_kernel<false><<<(n + 7) / 8, 256, 0, st>>>(layer, latent, idx_key, slot, swa_slot, n, ws, nullptr,
+                                                       nullptr);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_kv_norm_rope_pack(const csa_kv_layer &layer, const uint16_t *latent, const float *norm_w,
+                                     const float *rope_cs, const uint16_t *idx_key, const int64_t *slot,
+                                     const int32_t *swa_slot, int n, void *ws, cudaStream_t st)
+{
+    if (n == 0) return cudaSuccess;
+    kv_pack_kernel<true><<<(n + 7) / 8, 256, 0, st>>>(layer, latent, idx_key, slot, swa_slot, n, ws, norm_w,
+                                                      rope_cs);
     return cudaGetLastError();
 }
 

@@ -118,6 +118,25 @@ csa_status csa_kv_pack_fp4(const csa_kv_layer *layer, const uint16_t *latent,
                            int32_t n, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * Step 1 from the pre-norm latent -- RMSNorm, RoPE, then the pack of csa_kv_pack_fp4 ([ailily] 三:
+ * the latent is RMS-normalised, with weights of magnitude about 1, and rotated by RoPE, which keeps
+ * its norm).  The pages give no arithmetic; this call fixes it, in binary32, in this order:
+ *   v = bf16 latent; per 16-channel group g, s_g = FMA chain of v_c^2 (c = 16g .. 16g+15) from 0;
+ *   for d = 16, 8, 4, 2, 1: s_g <- s_g + s_(g xor d); r = 1 / sqrt(s_0 / 512 + 1e-6) (correctly
+ *   rounded); y_c = (v_c * r) * norm_weight_c; for pair i = 0..31 of channels (448 + 2i, 449 + 2i):
+ *   (a, b) -> (a*cos_i - b*sin_i, a*sin_i + b*cos_i), each product and sum rounded on its own;
+ *   the latent that is packed is bf16(y) (round to nearest even).
+ *   latent_prenorm bf16 [n][512]; norm_weight float [512]; rope_cos_sin float [n][32][2] =
+ *   (cos_i, sin_i) of each token's rotation; idx_key, slot, swa_slot as for csa_kv_pack_fp4.
+ * Results are bit-for-bit defined for finite inputs; ws needs CSA_WORKSPACE_HEADER_BYTES.
+ */
+csa_status csa_kv_norm_rope_pack_fp4(const csa_kv_layer *layer, const uint16_t *latent_prenorm,
+                                     const float *norm_weight, const float *rope_cos_sin,
+                                     const uint16_t *idx_key, const int64_t *slot,
+                                     const int32_t *swa_slot, int32_t n, void *ws, size_t ws_bytes,
+                                     void *stream);
+
+/*
  * Steps 2-3, Full layer -- score every block of every sequence and select its Top-k
  * ([rebasdaily] 同一份笔记，多层一起用: a Full layer re-selects Top-K over the whole range; the
  * first Full layer's scan builds the 2,048 x 8 candidate pool).
