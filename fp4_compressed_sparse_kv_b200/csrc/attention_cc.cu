@@ -13,6 +13,7 @@
 // in 8-position chunks) cut into `splits` contiguous ranges.  Each split writes an unnormalised
 // partial (o, m, l) that attn_combine_kernel merges.
 #include "attention_common.cuh"
+#include "pipeline.cuh"
 
 namespace csa {
 
@@ -206,6 +207,7 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const float *__restri
     __shared__ float wgt[kCombineMaxSplits];
     __shared__ float red[8];
     const int h = blockIdx.x, b = blockIdx.y, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    grid_dep_wait();   // every split's partial
     const float2 *ml = part_ml + (size_t)b * splits * H + h;
     float M = -INFINITY;
     for (int s = t; s < splits; s += 128) M = fmaxf(M, ml[(size_t)s * H].x);
@@ -261,9 +263,8 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const float *__restri
 cudaError_t launch_attn_combine(const AttnArgs &a, float *out, float *lse, cudaStream_t st)
 {
     dim3 grid(a.H, a.B);
-    attn_combine_kernel<<<grid, 128, 0, st>>>(a.part_o, reinterpret_cast<const float2 *>(a.part_ml), a.splits, a.H,
-                                              out, lse);
-    return cudaGetLastError();
+    return launch_overlapped(attn_combine_kernel, grid, dim3(128), 0, st, a.part_o,
+                             reinterpret_cast<const float2 *>(a.part_ml), a.splits, a.H, out, lse);
 }
 
 }  // namespace csa

@@ -278,15 +278,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_split_tc_kernel(AttnArgs a
     TcMisc &ms = *reinterpret_cast<TcMisc *>(base + kOffMisc);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    grid_dep_wait();   // the selected blocks of the previous grid
+    grid_dep_launch();   // the combine may be scheduled as splits finish
     const int s = blockIdx.x, b = blockIdx.y / head_groups, hg = blockIdx.y % head_groups;
     const int h0 = hg * kTcHeads;
-
-    SeqView sv;
-    const bool seq_ok = seq_view(a, b, sv);
-    int u_begin = 0, u_end = 0;
-    if (seq_ok) split_range(sv.units, s, a.splits, u_begin, u_end);
-    const int ntiles = (u_end - u_begin + kTcUnits - 1) / kTcUnits;
 
     if (threadIdx.x == 0) {
         mbar_init(&ms.s_full, 1);
@@ -301,6 +295,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_split_tc_kernel(AttnArgs a
     }
     if (threadIdx.x < kTcHeads) ms.m[threadIdx.x] = -INFINITY;
     if (threadIdx.x < 32) reinterpret_cast<uint32_t *>(ONES)[threadIdx.x] = 0x3C003C00u;   // fp16 1.0 pairs
+    __syncthreads();
+    // Q is an input of the step, not a result of the previous grid: load it while that grid finishes
+    if (warp < 8) load_q(a, ms, Q, b, h0, threadIdx.x);
+    grid_dep_wait();   // the selected blocks of the previous grid
+
+    SeqView sv;
+    const bool seq_ok = seq_view(a, b, sv);
+    int u_begin = 0, u_end = 0;
+    if (seq_ok) split_range(sv.units, s, a.splits, u_begin, u_end);
+    const int ntiles = (u_end - u_begin + kTcUnits - 1) / kTcUnits;
     if (warp == 8 && ntiles > 0) {
         tc_alloc(smem_addr(&ms.tmem_base), kTmemCols);
         tc_relinquish();
@@ -380,7 +384,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_split_tc_kernel(AttnArgs a
         const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
         TileRows rows;
         rows.load(a, sv, u_begin, u_end, 0, e, grp);
-        load_q(a, ms, Q, b, h0, threadIdx.x);
         if (grp == 0) ms.vmeta[0][e] = rows.valid ? 1.f : -1.f;
         bool ok = dequant_group(ms, V, rows, a, 0, e, grp);
         ok = warp_wait(&ms.q_ready, 0, &ms.abort_flag, a.ws, 1) && ok;   // every head's score scale
