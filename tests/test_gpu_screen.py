@@ -187,10 +187,11 @@ def test_screened_equals_exhaustive_exact_scan():
 
 
 @pytest.mark.parametrize("layout", ["sampled_high", "sampled_low"])
-def test_sampled_thresholds_fall_back_when_the_sample_misleads(layout):
-    """5,000 blocks, k = 3,000: the classification's strided sample (4,096 of the blocks) sees only
-    large-score blocks, or only small-score ones, so its threshold guesses fail their exact count
-    check and the exact radix selections must take over; the result still equals the oracle's."""
+def test_large_k_over_interleaved_magnitudes(layout):
+    """5,000 blocks, k = 3,000, large-score and small-score blocks interleaved on a fixed stride (4,096
+    of the blocks on one side, the rest on the other): the threshold bins of the lower bounds fall in
+    a crowded part of the distribution and thousands of blocks are sure; the selection still equals
+    the oracle's."""
     rng = np.random.default_rng([14, len(layout)])
     n, m, k = 5000, 4096, 3000
     sampled = np.zeros(n, bool)
