@@ -523,8 +523,11 @@ def run_reference(args, rank, world):
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": UNIT, "n_gpus": world,
             "steps": len(times), "warmup": args.warmup, "ms_per_step": round(1e3 * s / len(times), 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 attention, f32 indexer",
-            "data": "synthetic (seeded)", "config": {"workload": args.workload, "batch_per_gpu": 1,
-                                                     "seq_len": w.seq_lens[0], "heads": w.heads},
+            "data": "synthetic (seeded)",
+            # the workload of the other arm; each timed step is the bounded sample named in cpu_baseline
+            "config": {"workload": args.workload, "batch_per_gpu": w.batch, "seq_len": max(w.seq_lens),
+                       "heads": w.heads, "topk_blocks": w.topk, "modes": w.modes,
+                       "l2": "not applicable (host)", "parallelism": "dp%d replicas" % world},
             "cpu_baseline": {"value": round(value, 5), "unit": UNIT, "cores": 1, "kind": "oracle",
                              "sample": sample, "cpu": model, "host_cpus": ncpu},
             "e2e": {"value": round(value, 5), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
