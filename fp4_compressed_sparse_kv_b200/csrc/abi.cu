@@ -38,6 +38,7 @@ cudaError_t launch_finalize(const float *scores, int score_stride, const csa_bat
                             int32_t *out_blocks, int32_t *out_count, void *ws, cudaStream_t st);
 cudaError_t launch_attn_tc(const AttnArgs &a, cudaStream_t st);
 bool attn_tc_supported(int H);
+bool attn_tc_layer_ok(int num_pages, int num_rows);
 int attn_units_per_tile(int H);
 
 }  // namespace csa
@@ -296,6 +297,7 @@ csa_status csa_sparse_decode_attn(const csa_kv_layer *layer, const csa_batch *ba
         return CSA_ERR_INVALID_ARG;
     if (cap < 1 || cap > CSA_MAX_TOPK) return CSA_ERR_INVALID_ARG;
     if (!heads_ok(H)) return CSA_ERR_UNSUPPORTED;
+    if (attn_tc_supported(H) && !attn_tc_layer_ok(layer->num_pages, layer->num_rows)) return CSA_ERR_UNSUPPORTED;
     if (!(sm_scale > 0.f) || sm_scale > 1e30f) return CSA_ERR_INVALID_ARG;
     const WsLayout w = layout_for(batch->B, H, batch->max_seq_len, cap);
     if (ws_bytes < w.total) return CSA_ERR_WORKSPACE;

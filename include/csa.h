@@ -237,7 +237,8 @@ csa_status csa_index_reuse(int32_t B, const int32_t *prev_blocks, const int32_t 
  * e4m3 * swa_scale.  A position in both segments counts once in each.  z = tau * q_h . value;
  * out_h = softmax-weighted sum of values; lse_h = log-sum-exp of z.  Computed with fp16 operands
  * (exact for these values) and fp32 accumulation; agrees with exact arithmetic to within
- * 2e-3 of max|out| per sequence.
+ * 2e-3 of max|out| per sequence.  With H = 64 or 128 the caches may hold at most 2^31 FP4 entries
+ * (num_pages * 64) and 2^30 window entries (num_rows * 128); larger layers return CSA_ERR_UNSUPPORTED.
  */
 csa_status csa_sparse_decode_attn(const csa_kv_layer *layer, const csa_batch *batch,
                                   const uint16_t *q, int32_t H, float sm_scale,
@@ -284,10 +285,12 @@ csa_status csa_decode_layer(const csa_kv_layer *layer, const csa_batch *batch,
  * Limit: 256 + 4 * B * max(ceil(max_seq_len / 8), k) bytes must fit in CSA_NOALLOC_SCRATCH_BYTES
  * (4 MiB; e.g. 8 sequences of 131,072 tokens use 512 KiB); larger calls return CSA_ERR_WORKSPACE.
  * Every GPU that loads the library holds that array until the process exits.  The first call on each
- * device looks up the array's device address (cudaGetSymbolAddress, with that device current); make
- * that first call before any stream capture.  All calls on a device share the one array and each call
- * overwrites it: calls that overlap on the GPU (different streams without ordering between them) race
- * and give undefined results.  No allocation or free happens in any call.
+ * device looks up the array's device address (cudaGetSymbolAddress, with that device current) and keeps
+ * it for the life of the process; make that first call before any stream capture, and do not reset the
+ * device (cudaDeviceReset, or a primary-context reset) after it, since the kept address would then be
+ * stale.  All calls on a device share the one array and each call overwrites it: calls that overlap
+ * on the GPU (different streams without ordering between them) race and give undefined results.  No
+ * allocation or free happens in any call.
  */
 #define CSA_NOALLOC_SCRATCH_BYTES (4 << 20)
 csa_status csa_indexer_full_noalloc(const csa_kv_layer *layer, const csa_batch *batch,
