@@ -14,24 +14,25 @@
 // in fp32 on the CUDA cores from the unrounded probabilities (at most 2^-12 relative apart from the
 // fp16 numerators).
 //
-// Tile = 128 entries.  Both MMAs put the entries / channels on M = 128 ("swap AB"):
-//   QK:  S^T[128 entries x 64 heads]  = V[128 x 512] . Q^T               (A = V K-major, B = Q K-major)
-//   PV:  O^T[128 ch x 64 heads] (x4)  = V^T[128 ch x 128 entries] . P^T  (A = V^T MN-major, B = P^T MN-major)
-// One 128-byte-swizzled fp16 copy of the tile in shared memory is read as K-major V by QK and as
-// MN-major V^T by PV.  TMEM: O^T in 4 x 64 columns, S^T as two partial accumulators (even and odd
-// chunks, one per QK issuer, summed by the softmax) in 2 x 64 columns, and each row's softmax sums
-// in 64 columns.
+// Work unit: a half-tile of 64 entries.  Two half-tiles are in flight, each with its own V and P
+// buffer, so the dequantisation of one overlaps the MMAs and the softmax of the other.
+//   QK:  S^T[64 entries x 64 heads] = V[64 x 512] . Q^T        (M = 64; A = V K-major, B = Q K-major)
+//   PV:  O^T[128 ch x 64 heads] (x4) += V^T[128 ch x 64 entries] . P^T  (A = V^T MN-major, B = P^T MN-major)
+// The same 128-byte-swizzled fp16 copy of a half-tile is read as K-major V by QK and as MN-major V^T
+// by PV.  TMEM: O^T in 4 x 64 columns; S^T as four partial accumulators (one per MMA issuer, summed
+// by the softmax) in 4 x 64 columns, an M=64 accumulator taking 16 lanes of every 32: half-tile t
+// in the lower 16 lanes of each quarter when t is even, the upper 16 when odd.
 //
-// Warp roles (640 threads).  Warps 16-19 issue the MMAs (lane 0 each; warp 16 also owns the TMEM
-// allocation): one thread issues a tcgen05.mma only every ~100 cycles, so QK of the even and of the
-// odd chunks and PV of M-tiles 0-1 and 2-3 each have their own issuer.  Warps 0-15 form four groups of
-// four warps; thread e of a group is tile row e (TMEM lane e).  Group g owns heads 16g .. 16g+15 of
-// the softmax and channels 128g + e of the epilogue.  The V buffer is single; as PV(t) releases
-// M-tile m (V chunks 2m, 2m+1), all 512 threads dequantise those 128 channels of tile t+1 (thread
-// (g, e): 32 channels of entry e), from raw bytes loaded into registers a tile earlier.  Entry
-// addresses come from a table in shared memory that all threads fill after the grid dependency
-// (16 tiles at a time), so no dependent global load stalls a tile.  Softmax rescales lazily: O^T is
-// rescaled in TMEM only when a head's running maximum grows by more than 2^8.
+// Warp roles (640 threads).
+//   warps 0-7   producers: thread (e, cp) dequantises channels 128cp .. 128cp+127 of entry e from raw
+//               bytes it loaded two half-tiles earlier, once PV has released the buffer;
+//   warps 8-15  softmax: two groups of four warps, heads 32s .. 32s+31; a warp reads the 16 score rows
+//               of its TMEM quarter with 16-lane loads (thread t: rows t/4 and t/4+8, 8 heads);
+//   warps 16-19 MMA issuers (lane 0; warp 16 also owns the TMEM allocation).  One thread issues a
+//               tcgen05.mma only every ~100 cycles, longer than these MMAs take, so issuer r does QK
+//               of chunks r and r+4 (into S partial r) and PV of M-tile r, QK one half-tile ahead.
+// Softmax rescales lazily: O^T is rescaled in TMEM only when a head's running maximum grows by more
+// than 2^8 (after waiting for the previous half-tile's PV).
 #include "attention_common.cuh"
 #include "pipeline.cuh"
 #include "tcgen05.cuh"
@@ -39,26 +40,27 @@
 namespace csa {
 
 constexpr int kTcHeads = 64;
-constexpr int kTcRows = 128;
-constexpr int kTcUnits = kTcRows / kAttnUnit;    // 16 units of 8 entries per tile
+constexpr int kHalf = 64;                        // entries per half-tile
+constexpr int kHalfUnits = kHalf / kAttnUnit;    // 8 units of 8 entries
+constexpr int kTcUnits = 2 * kHalfUnits;         // units per 128-entry tile (split sizing)
 constexpr int kTcChunks = kLatent / 64;          // 8 chunks of 64 channels
-constexpr int kTcGroups = 4;                     // compute groups of 4 warps
-constexpr int kTcHeadsPerGroup = kTcHeads / kTcGroups;
-constexpr int kTcIssuers = 4;                    // MMA-issuing warps: QK even / odd chunks, PV M-tiles 0-1 / 2-3
-constexpr int kTcThreads = 32 * (4 * kTcGroups + kTcIssuers);
-constexpr int kTcCompute = 128 * kTcGroups;
-constexpr int kSAcc = 2;
-constexpr int kTabTiles = 16;                    // tiles of entry addresses resolved at a time                         // partial QK accumulators (independent MMA chains)
-constexpr uint32_t kVChunk = kTcRows * 128;      // 16 KB: 128 rows x 64 fp16
+constexpr int kProducers = 256;                  // warps 0-7
+constexpr int kSoftmax = 256;                    // warps 8-15
+constexpr int kTcThreads = 640;
+constexpr int kTcCompute = kProducers + kSoftmax;
+constexpr uint32_t kVChunk = kHalf * 128;        // 8 KB: 64 rows x 64 fp16
+constexpr uint32_t kVBuf = kTcChunks * kVChunk;  // 64 KB per half-tile buffer
 constexpr uint32_t kQChunk = kTcHeads * 128;     // 8 KB: 64 rows x 64 fp16
+constexpr uint32_t kPBuf = kHalf * 128;          // 8 KB: 64 entry rows x 64 heads fp16
+constexpr int kTabHalves = 32;                   // half-tiles of entry addresses resolved at a time
 constexpr uint32_t kOffV = 0;
-constexpr uint32_t kOffQ = kOffV + kTcChunks * kVChunk;
+constexpr uint32_t kOffQ = kOffV + 2 * kVBuf;
 constexpr uint32_t kOffP = kOffQ + kTcChunks * kQChunk;
-constexpr uint32_t kOffMisc = kOffP + kTcRows * 128;
+constexpr uint32_t kOffTab = kOffP + 2 * kPBuf;
+constexpr uint32_t kOffMisc = kOffTab + kTabHalves * kHalf * 4;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0;                    // O^T: M-tile m in columns 64m .. 64m+63
-constexpr uint32_t kColS = 256;                  // S^T partial a in columns 256 + 64a ..
-constexpr uint32_t kColL = kColS + 64 * kSAcc;   // per-row softmax sums: group g in 16 columns at 16g
+constexpr uint32_t kColS = 256;                  // S^T partial r in columns 256 + 64r ..
 constexpr float kLazy = 8.f;      // log2-domain growth of a head maximum tolerated without rescaling
 constexpr float kPOffset = 7.f;   // p = exp2(z - m + 7) <= 2^15 keeps small p out of fp16 subnormals
 constexpr float kNoMax = -1e30f;  // running maximum before any finite score (exp2 of it minus a finite value is 0)
@@ -66,25 +68,23 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
 struct TcMisc {
-    uint64_t s_full, p_full, q_ready, o_done;
-    uint64_t final_bar[kTcIssuers];
-    uint64_t v_ready[4];          // per PV M-tile: its 128 channels of the next tile are written
-    uint64_t v_free[4];           // per PV M-tile: PV has finished reading them
+    uint64_t q_ready, o_done;
+    uint64_t v_ready[2], v_free[2], s_full[2], p_full[2];
+    uint64_t final_bar[4];
     uint32_t tmem_base;
     int abort_flag;
-    float qmax[16];                              // per compute warp: largest |q| of its rows
-    float red[kTcGroups][4][kTcHeadsPerGroup];   // per group, per warp: a per-head partial
-    float mx[kTcGroups][kTcHeadsPerGroup];       // running maximum of each head (log2 domain)
-    int32_t rows[kTabTiles][kTcRows];            // entry of (tile, row): FP4 cache row >= 0, window slot
-                                                 // -(slot + 2), or -1 (masked)
-    float alpha[kTcGroups][kTcHeadsPerGroup];    // rescale factor of each head at a maximum update
-    SeqView sv;                                  // the sequence, read from here by every thread
     int u_begin, u_end;                          // this split's units
+    SeqView sv;                                  // the sequence, read from here by every thread
+    float qmax[16];                              // per Q-loading warp: largest |q| of its rows
+    float mx[kTcHeads];                          // running maximum of each head (log2 domain)
+    float alpha[kTcHeads];                       // rescale factor of each head at a maximum update
+    float red[2][4][32];                         // per softmax group and warp: a per-head partial
+    uint64_t vmask[2];                           // valid rows of the half-tile in each V buffer
 };
 
 constexpr size_t kTcSmem = kOffMisc + sizeof(TcMisc) + 1024;
 
-constexpr uint32_t kIdescQK = umma_idesc_f16(128, kTcHeads, false, false);
+constexpr uint32_t kIdescQK = umma_idesc_f16(64, kTcHeads, false, false);
 constexpr uint32_t kIdescPV = umma_idesc_f16(128, kTcHeads, true, true);
 
 __device__ __forceinline__ uint32_t swz(uint32_t row, uint32_t unit) { return row * 128u + ((unit ^ (row & 7u)) << 4); }
@@ -102,34 +102,50 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi)
     return *reinterpret_cast<uint32_t *>(&h);
 }
 
-// Group barriers (named barrier `id` over the 128 threads of one group).  Every thread of the group
-// executes each of them once per tile, also after a failed wait, so none can be left waiting.
-__device__ __forceinline__ bool group_and(int id, bool v)
+// Named barriers: 1, 2 = the two softmax groups (128 threads each); 3 = the producers (256);
+// 4 = producers and softmax warps (512).  Every participant executes each of them the same number of
+// times, also after a failed wait.
+__device__ __forceinline__ bool bar_and(int id, int n, bool v)
 {
     int r;
-    asm volatile("{\n.reg .pred p, q;\nsetp.ne.b32 q, %2, 0;\nbar.red.and.pred p, %1, 128, q;\nselp.b32 %0, 1, 0, p;\n}"
+    asm volatile("{\n.reg .pred p, q;\nsetp.ne.b32 q, %3, 0;\nbar.red.and.pred p, %1, %2, q;\nselp.b32 %0, 1, 0, p;\n}"
                  : "=r"(r)
-                 : "r"(id), "r"((int)v)
+                 : "r"(id), "r"(n), "r"((int)v)
                  : "memory");
     return r != 0;
 }
 
-__device__ __forceinline__ bool group_or(int id, bool v)
+__device__ __forceinline__ bool bar_or(int id, int n, bool v)
 {
     int r;
-    asm volatile("{\n.reg .pred p, q;\nsetp.ne.b32 q, %2, 0;\nbar.red.or.pred p, %1, 128, q;\nselp.b32 %0, 1, 0, p;\n}"
+    asm volatile("{\n.reg .pred p, q;\nsetp.ne.b32 q, %3, 0;\nbar.red.or.pred p, %1, %2, q;\nselp.b32 %0, 1, 0, p;\n}"
                  : "=r"(r)
-                 : "r"(id), "r"((int)v)
+                 : "r"(id), "r"(n), "r"((int)v)
                  : "memory");
     return r != 0;
 }
 
-__device__ __forceinline__ void group_sync(int id) { asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory"); }
+__device__ __forceinline__ void bar_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 
-// Barrier over the 512 compute threads (the MMA warp does not take part).
-__device__ __forceinline__ void compute_sync() { asm volatile("bar.sync 5, %0;" ::"n"(kTcCompute) : "memory"); }
+// 16 lanes x (4 x 8) columns: thread t gets rows t/4 and t/4 + 8 of the 16 lanes at taddr, columns
+// 8j + 2(t%4) and 8j + 2(t%4) + 1 for j = 0..3: v[4j] (row t/4, even column), v[4j+1] (row t/4, odd),
+// v[4j+2], v[4j+3] (row t/4 + 8).  Waited for in the same statement.
+__device__ __forceinline__ void tc_ld16x256_x4_sync(uint32_t taddr, float *v)
+{
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
 
-// 32 lanes x 16 consecutive 32-bit columns, waited for in the same statement.
+// 32 lanes x 16 consecutive 32-bit columns (thread i: lane i), waited for in the same statement.
 __device__ __forceinline__ void tc_ld16_sync(uint32_t taddr, float *v)
 {
     uint32_t r[16];
@@ -159,143 +175,140 @@ __device__ __forceinline__ void tc_st16(uint32_t taddr, const float *v)
         : "memory");
 }
 
-// This thread's row of the group's 16 scores in the log2 domain: the sum of the partial QK
-// accumulators times zs; a masked row gives -inf.
-__device__ __forceinline__ void load_scores(uint32_t taddr, bool valid, float zs, float *z)
+// Half-tile-aligned split of a sequence's units: split s of `splits` gets whole 8-unit half-tiles,
+// so every half-tile but the sequence's last is full.
+__device__ __forceinline__ void split_halves(int units, int s, int splits, int &ub, int &ue)
 {
-    tc_ld16_sync(taddr, z);
-#pragma unroll
-    for (int aa = 1; aa < kSAcc; ++aa) {
-        float z2[kTcHeadsPerGroup];
-        tc_ld16_sync(taddr + 64 * aa, z2);
-#pragma unroll
-        for (int q = 0; q < kTcHeadsPerGroup; ++q) z[q] += z2[q];
-    }
-#pragma unroll
-    for (int q = 0; q < kTcHeadsPerGroup; ++q) z[q] = valid ? z[q] * zs : -INFINITY;
+    const int halves = (units + kHalfUnits - 1) / kHalfUnits;
+    const int hb = (int)((long long)halves * s / splits), he = (int)((long long)halves * (s + 1) / splits);
+    ub = hb * kHalfUnits;
+    ue = he * kHalfUnits < units ? he * kHalfUnits : units;
 }
 
-// Tile-aligned split of a sequence's units: split s of `splits` gets whole 16-unit tiles, so every
-// tile but the sequence's last is full.
-__device__ __forceinline__ void split_tiles(int units, int s, int splits, int &ub, int &ue)
-{
-    const int tiles = (units + kTcUnits - 1) / kTcUnits;
-    const int tb = (int)((long long)tiles * s / splits), te = (int)((long long)tiles * (s + 1) / splits);
-    ub = tb * kTcUnits;
-    ue = te * kTcUnits < units ? te * kTcUnits : units;
-}
+// Entry table: for each row e of each half-tile, the FP4 cache row (page * 64 + offset) of the entry,
+// -(slot + 2) for a window entry, or -1 for a masked row (past the split or the sequence).
 
-// Table code of (tile t, row e) of this split: the FP4 cache row (page * 64 + offset) of the entry,
-// -(slot + 2) for a window entry, -1 for a masked row (past the split or the sequence).
-__device__ __forceinline__ int32_t entry_code(const AttnArgs &a, const SeqView &sv, int u_begin, int u_end, int t, int e)
-{
-    const int u = u_begin + t * kTcUnits + e / kAttnUnit, j = e % kAttnUnit;
-    if (u >= u_end) return -1;
-    if (u < sv.nE) {
-        const int blk = sv.blocks[u];
-        if (blk < 0 || blk >= sv.nb) {
-            report(a.ws, CSA_ERR_DEVICE_DATA, u);
-            return -1;
-        }
-        const int p = blk * kBlock + j;
-        if (p >= sv.L) return -1;
-        const int page = sv.bt[blk / kBlocksPerPage];
-        if (page < 0 || page >= a.num_pages) {
-            report(a.ws, CSA_ERR_DEVICE_DATA, blk);
-            return -1;
-        }
-        return page * kPage + (blk % kBlocksPerPage) * kBlock + j;
-    }
-    const int p = sv.w0 + (u - sv.nE) * kAttnUnit + j;
-    if (p >= sv.L) return -1;
-    return -(sv.row * kWindow + (p % kWindow) + 2);
-}
-
-// One thread's share of one tile: entry e, and in each M-tile m the 32 channels 128m + 32g .. +31.
-// The raw bytes of an FP4 entry (16 B of codes and 2 scale bytes per M-tile) are loaded into
-// registers a tile before they are dequantised; a window entry (32 E4M3 values per M-tile) is read
-// when it is written, since the window is at most one tile of a sequence.
-struct RawTile {
+// A producer thread's share of one half-tile: entry e, channels 128cp .. 128cp+127 (V chunks 2cp,
+// 2cp+1).  The raw bytes of an FP4 entry (64 B of codes, 8 scale bytes, contiguous) are loaded
+// into registers two half-tiles before they are dequantised; a window entry (128 E4M3 values) is
+// read when it is written, since the window is at most two half-tiles of a sequence.  (A mapping in
+// which one warp-wide load covers two whole entries loads fewer lines but writes the swizzled
+// V rows with 4-way bank conflicts, which costs more.)
+struct RawHalf {
     uint4 code[4];
-    uint32_t sc[4];
+    uint2 sc;
     int32_t row;
 
-    __device__ __forceinline__ void fetch(const AttnArgs &a, int32_t code_row, int g)
+    __device__ __forceinline__ void fetch(const AttnArgs &a, int32_t code_row, int cp)
     {
         row = code_row;
         if (row >= 0) {
-            const uint8_t *cp = a.codes + (size_t)row * kCodeBytes + 16 * g;
-            const uint8_t *sp = a.scales + (size_t)row * kScaleBytes + 2 * g;
+            const uint4 *cp4 = reinterpret_cast<const uint4 *>(a.codes + (size_t)row * kCodeBytes + 64 * cp);
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                code[m] = *reinterpret_cast<const uint4 *>(cp + 64 * m);
-                sc[m] = *reinterpret_cast<const uint16_t *>(sp + 8 * m);
-            }
+            for (int q = 0; q < 4; ++q) code[q] = cp4[q];
+            sc = *reinterpret_cast<const uint2 *>(a.scales + (size_t)row * kScaleBytes + 8 * cp);
         }
     }
 
-    // Dequantise this thread's 32 channels of M-tile m (V chunk 2m + g/2, 16-byte units 4(g%2) ..
-    // 4(g%2)+3 of row e).
-    __device__ __forceinline__ void write(const AttnArgs &a, uint8_t *V, int m, int e, int g) const
+    // Dequantise into V chunks 2cp + h (h = 0, 1), row e.
+    __device__ __forceinline__ void write(const AttnArgs &a, uint8_t *Vb, int e, int cp) const
     {
-        uint8_t *dst = V + (2 * m + (g >> 1)) * kVChunk;
-        const uint32_t u0 = 4u * (uint32_t)(g & 1);
-        if (row == -1) {
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj)
-                *reinterpret_cast<uint4 *>(dst + swz((uint32_t)e, u0 + jj)) = make_uint4(0u, 0u, 0u, 0u);
-        } else if (row >= 0) {
+        for (int h = 0; h < 2; ++h) {
+            uint8_t *dst = Vb + (2 * cp + h) * kVChunk;
+            if (row == -1) {
 #pragma unroll
-            for (int gg = 0; gg < 2; ++gg) {
-                const uint32_t sh = e4m3x2_to_f16x2((uint16_t)((sc[m] >> (8 * gg)) & 0xFF));
-                const uint32_t s2 = (sh & 0xFFFFu) | (sh << 16);
-                const uint32_t w0 = gg ? code[m].z : code[m].x, w1 = gg ? code[m].w : code[m].y;
-                uint32_t v[8];
+                for (int jj = 0; jj < 8; ++jj)
+                    *reinterpret_cast<uint4 *>(dst + swz((uint32_t)e, (uint32_t)jj)) = make_uint4(0u, 0u, 0u, 0u);
+            } else if (row >= 0) {
+                const uint32_t sw = h ? sc.y : sc.x;
+#pragma unroll
+                for (int gg = 0; gg < 4; ++gg) {
+                    const uint32_t sh = e4m3x2_to_f16x2((uint16_t)((sw >> (8 * gg)) & 0xFF));
+                    const uint32_t s2 = (sh & 0xFFFFu) | (sh << 16);
+                    const uint4 cw = code[2 * h + (gg >> 1)];
+                    const uint32_t w0 = (gg & 1) ? cw.z : cw.x, w1 = (gg & 1) ? cw.w : cw.y;
+                    uint32_t v[8];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        v[q] = hmul2_u32(e2m1x2_to_f16x2((uint8_t)(w0 >> (8 * q))), s2);
+                        v[4 + q] = hmul2_u32(e2m1x2_to_f16x2((uint8_t)(w1 >> (8 * q))), s2);
+                    }
+                    *reinterpret_cast<uint4 *>(dst + swz((uint32_t)e, (uint32_t)(2 * gg))) =
+                        make_uint4(v[0], v[1], v[2], v[3]);
+                    *reinterpret_cast<uint4 *>(dst + swz((uint32_t)e, (uint32_t)(2 * gg + 1))) =
+                        make_uint4(v[4], v[5], v[6], v[7]);
+                }
+            } else {
+                // window entry: 64 E4M3 values times the entry's binary32 scale, rounded to fp16
+                const size_t slot = (size_t)(-row - 2);
+                const float fs = a.swa_scale[slot];
+                const uint4 *src = reinterpret_cast<const uint4 *>(a.swa + slot * kLatent + 128 * cp + 64 * h);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    v[q] = hmul2_u32(e2m1x2_to_f16x2((uint8_t)(w0 >> (8 * q))), s2);
-                    v[4 + q] = hmul2_u32(e2m1x2_to_f16x2((uint8_t)(w1 >> (8 * q))), s2);
-                }
-                *reinterpret_cast<uint4 *>(dst + swz((uint32_t)e, u0 + 2 * gg)) = make_uint4(v[0], v[1], v[2], v[3]);
-                *reinterpret_cast<uint4 *>(dst + swz((uint32_t)e, u0 + 2 * gg + 1)) = make_uint4(v[4], v[5], v[6], v[7]);
-            }
-        } else {
-            // window entry: 32 E4M3 values times the entry's binary32 scale, rounded to fp16
-            const size_t slot = (size_t)(-row - 2);
-            const float fs = a.swa_scale[slot];
-            const uint4 *src = reinterpret_cast<const uint4 *>(a.swa + slot * kLatent + 128 * m + 32 * g);
+                    const uint4 w = src[q];
+                    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+                    uint32_t v[8];
 #pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                const uint4 w = src[q];
-                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-                uint32_t v[8];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const uint32_t lo = e4m3x2_to_f16x2((uint16_t)(ww[k] & 0xFFFF));
-                    const uint32_t hi = e4m3x2_to_f16x2((uint16_t)(ww[k] >> 16));
-                    v[2 * k] = pack_f16x2(h_lo(lo) * fs, h_hi(lo) * fs);
-                    v[2 * k + 1] = pack_f16x2(h_lo(hi) * fs, h_hi(hi) * fs);
+                    for (int k = 0; k < 4; ++k) {
+                        const uint32_t lo = e4m3x2_to_f16x2((uint16_t)(ww[k] & 0xFFFF));
+                        const uint32_t hi = e4m3x2_to_f16x2((uint16_t)(ww[k] >> 16));
+                        v[2 * k] = pack_f16x2(h_lo(lo) * fs, h_hi(lo) * fs);
+                        v[2 * k + 1] = pack_f16x2(h_lo(hi) * fs, h_hi(hi) * fs);
+                    }
+                    *reinterpret_cast<uint4 *>(dst + swz((uint32_t)e, (uint32_t)(2 * q))) = make_uint4(v[0], v[1], v[2], v[3]);
+                    *reinterpret_cast<uint4 *>(dst + swz((uint32_t)e, (uint32_t)(2 * q + 1))) =
+                        make_uint4(v[4], v[5], v[6], v[7]);
                 }
-                *reinterpret_cast<uint4 *>(dst + swz((uint32_t)e, u0 + 2 * q)) = make_uint4(v[0], v[1], v[2], v[3]);
-                *reinterpret_cast<uint4 *>(dst + swz((uint32_t)e, u0 + 2 * q + 1)) = make_uint4(v[4], v[5], v[6], v[7]);
             }
         }
     }
 };
 
-// Fill the entry table with tiles t0 .. t0 + kTabTiles - 1 (every compute thread takes a share).
-__device__ __forceinline__ void fill_table(const AttnArgs &a, TcMisc &ms, int t0, int ntiles, int tid)
+// Fill the entry table with half-tiles t0 .. t0 + kTabHalves - 1: producer thread i takes unit i of
+// the range (8 entries: one selected block, or 8 window positions), so the block id and the page
+// table are read once per unit, in two rounds of independent loads.
+static_assert(kTabHalves * kHalfUnits == kProducers, "one unit of the table per producer thread");
+__device__ __forceinline__ void fill_table(const AttnArgs &a, TcMisc &ms, int32_t *tab, int t0, int tid)
 {
-    const int n = (ntiles - t0 < kTabTiles ? ntiles - t0 : kTabTiles) * kTcRows;
-    for (int i = tid; i < n; i += kTcCompute)
-        ms.rows[i / kTcRows][i % kTcRows] = entry_code(a, ms.sv, ms.u_begin, ms.u_end, t0 + i / kTcRows, i % kTcRows);
+    const SeqView &sv = ms.sv;
+    const int u = ms.u_begin + t0 * kHalfUnits + tid;
+    int32_t *out = tab + tid * kAttnUnit;
+    int32_t code = -1;         // code of position 0 of the unit, or -1 for none
+    int limit = 0;             // positions j < limit of the unit are valid
+    if (u < ms.u_end) {
+        if (u < sv.nE) {
+            const int blk = sv.blocks[u];
+            if (blk < 0 || blk >= sv.nb) {
+                report(a.ws, CSA_ERR_DEVICE_DATA, u);
+            } else {
+                const int page = sv.bt[blk / kBlocksPerPage];
+                if (page < 0 || page >= a.num_pages) {
+                    report(a.ws, CSA_ERR_DEVICE_DATA, blk);
+                } else {
+                    code = page * kPage + (blk % kBlocksPerPage) * kBlock;
+                    limit = sv.L - blk * kBlock;
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < kAttnUnit; ++j) out[j] = (code >= 0 && j < limit) ? code + j : -1;
+        } else {
+            const int p0 = sv.w0 + (u - sv.nE) * kAttnUnit;
+#pragma unroll
+            for (int j = 0; j < kAttnUnit; ++j)
+                out[j] = (p0 + j < sv.L) ? -(sv.row * kWindow + ((p0 + j) % kWindow) + 2) : -1;
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < kAttnUnit; ++j) out[j] = -1;
+    }
 }
 
 // Q of heads h0..h0+63 into shared memory as fp16, 128B-swizzled K-major, scaled by one power of two
 // 2^k that puts the largest |q| of the 64 heads in [2^13, 2^14); returns tau * log2(e) * 2^-k, the
-// factor that turns an accumulated score into the log2 domain.  Compute thread t converts channels
-// 64(t/64) .. 64(t/64)+63 of head t%64 (consecutive threads write different rows of one chunk, so
-// the 16-byte stores do not collide in shared-memory banks).
+// factor that turns an accumulated score into the log2 domain.  Thread t (of the 512 producer and
+// softmax threads) converts channels 64(t/64) .. 64(t/64)+63 of head t%64 (consecutive threads write
+// different rows of one chunk, so the 16-byte stores do not collide in shared-memory banks).
 __device__ __forceinline__ float load_q(const AttnArgs &a, TcMisc &ms, uint8_t *Q, int b, int h0, int t)
 {
     const int h = t & 63, part = t >> 6;
@@ -313,7 +326,7 @@ __device__ __forceinline__ float load_q(const AttnArgs &a, TcMisc &ms, uint8_t *
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     if ((t & 31) == 0) ms.qmax[t >> 5] = amax;
-    compute_sync();
+    bar_sync(4, kTcCompute);
     amax = 0.f;
 #pragma unroll
     for (int w = 0; w < 16; ++w) amax = fmaxf(amax, ms.qmax[w]);
@@ -338,8 +351,24 @@ __device__ __forceinline__ float load_q(const AttnArgs &a, TcMisc &ms, uint8_t *
     return a.sm_scale * exp2f((float)-k) * kLog2e;
 }
 
-// M-tiles in the order PV releases them (issuer 2 does M-tile 0 then 1, issuer 3 M-tile 2 then 3).
-__device__ __forceinline__ int release_order(int i) { return (i & 1) * 2 + (i >> 1); }
+// This thread's 16 scores (rows t/4 and t/4 + 8 of its warp's quarter, 8 heads of its group) in the
+// log2 domain: the sum of the four partial accumulators times zs; a masked row gives -inf.
+__device__ __forceinline__ void load_scores(uint32_t taddr, bool v0, bool v1, float zs, float *z)
+{
+    tc_ld16x256_x4_sync(taddr, z);
+#pragma unroll
+    for (int r = 1; r < 4; ++r) {
+        float z2[16];
+        tc_ld16x256_x4_sync(taddr + 64 * r, z2);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) z[i] += z2[i];
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const bool valid = (i & 2) ? v1 : v0;
+        z[i] = valid ? z[i] * zs : -INFINITY;
+    }
+}
 
 __global__ void __launch_bounds__(kTcThreads, 1) attn_split_tc_kernel(AttnArgs a, int head_groups)
 {
@@ -348,6 +377,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_split_tc_kernel(AttnArgs a
     uint8_t *V = base + kOffV;
     uint8_t *Q = base + kOffQ;
     uint8_t *P = base + kOffP;
+    int32_t *tab = reinterpret_cast<int32_t *>(base + kOffTab);
     TcMisc &ms = *reinterpret_cast<TcMisc *>(base + kOffMisc);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -356,18 +386,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_split_tc_kernel(AttnArgs a
     const int h0 = hg * kTcHeads;
 
     if (threadIdx.x == 0) {
-        mbar_init(&ms.s_full, 2);     // both QK issuers
-        mbar_init(&ms.p_full, kTcCompute);
         mbar_init(&ms.q_ready, kTcCompute);
-        mbar_init(&ms.o_done, 2);     // both PV issuers
-        for (int r = 0; r < kTcIssuers; ++r) mbar_init(&ms.final_bar[r], 1);
-        for (int m = 0; m < 4; ++m) {
-            mbar_init(&ms.v_ready[m], kTcCompute);
-            mbar_init(&ms.v_free[m], 1);
+        mbar_init(&ms.o_done, 4);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&ms.v_ready[i], kProducers);
+            mbar_init(&ms.v_free[i], 4);
+            mbar_init(&ms.s_full[i], 4);
+            mbar_init(&ms.p_full[i], kSoftmax);
         }
+        for (int r = 0; r < 4; ++r) mbar_init(&ms.final_bar[r], 1);
         ms.abort_flag = 0;
         fence_mbar_init();
     }
+    if (threadIdx.x < kTcHeads) ms.mx[threadIdx.x] = kNoMax;
     __syncthreads();
     // Q is an input of the step, not a result of the previous grid: load it while that grid finishes
     float zs = 0.f;
@@ -376,24 +407,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_split_tc_kernel(AttnArgs a
 
     if (threadIdx.x == 0) {
         int ub = 0, ue = 0;
-        if (seq_view(a, b, ms.sv)) split_tiles(ms.sv.units, s, a.splits, ub, ue);
+        if (seq_view(a, b, ms.sv)) split_halves(ms.sv.units, s, a.splits, ub, ue);
         ms.u_begin = ub;
         ms.u_end = ue;
     }
     __syncthreads();
-    const int ntiles = (ms.u_end - ms.u_begin + kTcUnits - 1) / kTcUnits;
-    if (warp == 16 && ntiles > 0) {
+    const int nh = (ms.u_end - ms.u_begin + kHalfUnits - 1) / kHalfUnits;   // half-tiles of this split
+    if (warp == 16 && nh > 0) {
         tc_alloc(smem_addr(&ms.tmem_base), kTmemCols);
         tc_relinquish();
     }
-    if (warp < 16 && ntiles > 0) fill_table(a, ms, 0, ntiles, threadIdx.x);
+    if (warp < 8 && nh > 0) fill_table(a, ms, tab, 0, threadIdx.x);
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = ms.tmem_base;
 
-    if (ntiles == 0) {
+    if (nh == 0) {
         // empty split: a neutral partial
         if (warp < 4) {
             float *po = a.part_o + (((size_t)b * a.splits + s) * a.H + h0) * kLatent;
@@ -406,51 +437,76 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_split_tc_kernel(AttnArgs a
         return;
     }
 
+    bool ok = true;
     if (warp >= 16) {
         // ------------------------------- MMA issuers -------------------------------
-        // One thread issues a tcgen05.mma only every ~100 cycles, longer than an M=128, N=64, K=16
-        // MMA takes, so four warps issue: QK of the even chunks into S partial 0 and of the odd
-        // chunks into partial 1 (M-tile by M-tile as the dequantisation finishes them), and PV of
-        // M-tiles 0, 1 and of M-tiles 2, 3, one M-tile after the other so that the first two are
-        // released early.
         const int r = warp - 16;
         if (lane == 0) {
             const uint32_t sV = smem_addr(V), sQ = smem_addr(Q), sP = smem_addr(P);
-            bool ok = true;
-            if (r < 2) {
-                ok = mbar_wait(&ms.q_ready, 0, &ms.abort_flag, a.ws, 1);
-                for (int t = 0; ok && t < ntiles; ++t) {
-                    // S is read by every group's softmax of the previous tile
-                    if (t > 0 && !(ok = mbar_wait(&ms.p_full, (t - 1) & 1, &ms.abort_flag, a.ws, 3))) break;
-                    for (int i = 0; i < 4; ++i) {
-                        const int m = release_order(i);
-                        if (!(ok = mbar_wait(&ms.v_ready[m], t & 1, &ms.abort_flag, a.ws, 2))) break;
-                        tc_fence_after();
-                        const int c = 2 * m + r;
+            ok = mbar_wait(&ms.q_ready, 0, &ms.abort_flag, a.ws, 1);
+            tc_fence_after();
+            // QK of chunks r and r + 4 of half-tile t into S partial r, lanes of parity t % 2
+            auto issue_qk = [&](int t) {
+                const int p = t & 1;
+                const uint32_t dS = tmem + ((uint32_t)(16 * p) << 16) + kColS + 64 * r;
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            const uint64_t ad = umma_sdesc_sw128(sV + c * kVChunk + kk * 32, 16, 1024);
-                            const uint64_t bd = umma_sdesc_sw128(sQ + c * kQChunk + kk * 32, 16, 1024);
-                            tc_mma_f16(tmem + kColS + 64 * r, ad, bd, kIdescQK, (i > 0 || kk > 0) ? 1u : 0u);
-                        }
+                for (int i = 0; i < 2; ++i) {
+                    const int c = r + 4 * i;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t ad = umma_sdesc_sw128(sV + p * kVBuf + c * kVChunk + kk * 32, 16, 1024);
+                        const uint64_t bd = umma_sdesc_sw128(sQ + c * kQChunk + kk * 32, 16, 1024);
+                        tc_mma_f16(dS, ad, bd, kIdescQK, (i > 0 || kk > 0) ? 1u : 0u);
                     }
-                    if (!ok) break;
-                    tc_commit(smem_addr(&ms.s_full));
                 }
-            } else {
-                for (int t = 0; ok && t < ntiles; ++t) {
-                    if (!(ok = mbar_wait(&ms.p_full, t & 1, &ms.abort_flag, a.ws, 3))) break;
-                    tc_fence_after();
-                    for (int m = 2 * (r - 2); m < 2 * (r - 2) + 2; ++m) {
+                tc_commit(smem_addr(&ms.s_full[p]));
+            };
+            // PV of M-tile r of half-tile t
+            auto issue_pv = [&](int t) {
+                const int p = t & 1;
 #pragma unroll
-                        for (int kk = 0; kk < kTcRows / 16; ++kk) {
-                            const uint64_t ad = umma_sdesc_sw128(sV + 2 * m * kVChunk + kk * 2048, kVChunk, 1024);
-                            const uint64_t bd = umma_sdesc_sw128(sP + kk * 2048, kVChunk, 1024);
-                            tc_mma_f16(tmem + kColO + 64 * m, ad, bd, kIdescPV, (t > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < kHalf / 16; ++kk) {
+                    const uint64_t ad = umma_sdesc_sw128(sV + p * kVBuf + 2 * r * kVChunk + kk * 2048, kVChunk, 1024);
+                    const uint64_t bd = umma_sdesc_sw128(sP + p * kPBuf + kk * 2048, kVChunk, 1024);
+                    tc_mma_f16(tmem + kColO + 64 * r, ad, bd, kIdescPV, (t > 0 || kk > 0) ? 1u : 0u);
+                }
+                tc_commit(smem_addr(&ms.v_free[p]));
+                if (t == nh - 1) tc_commit(smem_addr(&ms.o_done));
+            };
+            // Issue whichever is ready first: PV(pv) once the softmax has written P(pv), QK(qk) once the
+            // producers have written half-tile qk, so that the chains of the even and of the odd
+            // half-tiles overlap.  (QK(t) precedes PV(t) through the softmax; QK(t+2) follows PV(t)
+            // through the producers, who wait for it before reusing the buffer.)  The waits are
+            // polled together, under the same limit as every other wait.
+            int qk = 0, pv = 0;
+            unsigned long long t0 = 0;
+            for (uint32_t it = 0; ok && pv < nh; ++it) {
+                if (pv < qk && mbar_try_wait(&ms.p_full[pv & 1], (pv >> 1) & 1)) {
+                    tc_fence_after();
+                    issue_pv(pv++);
+                    t0 = 0;
+                    continue;
+                }
+                if (qk < nh && mbar_try_wait(&ms.v_ready[qk & 1], (qk >> 1) & 1)) {
+                    tc_fence_after();
+                    issue_qk(qk++);
+                    t0 = 0;
+                    continue;
+                }
+                if ((it & 63u) == 0) {
+                    volatile int *abort_flag = &ms.abort_flag;
+                    if (*abort_flag) {
+                        ok = false;
+                    } else {
+                        const unsigned long long now = global_ns();
+                        if (t0 == 0) {
+                            t0 = now;
+                        } else if (now - t0 > kWaitLimitNs) {
+                            *abort_flag = 1;
+                            report(a.ws, CSA_ERR_TIMEOUT, 2);
+                            ok = false;
                         }
-                        tc_commit(smem_addr(&ms.v_free[m]));
                     }
-                    if (t == ntiles - 1) tc_commit(smem_addr(&ms.o_done));
                 }
             }
             // every MMA this thread issued has completed before TMEM is released
@@ -459,162 +515,179 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_split_tc_kernel(AttnArgs a
             mbar_wait(&ms.final_bar[r], 0, &no_abort, a.ws, 4);
         }
         __syncwarp();
-    } else {
-        // ------------------- compute groups: group g = warps 4g .. 4g+3 -------------------
-        const int g = warp >> 2;
-        const int bar_id = 1 + g;            // named barrier of the group
-        const int e = threadIdx.x & 127;     // TMEM lane = tile row (entry); channel in the epilogue
-        const int wq = warp & 3;
-        const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
-        const int hb = kTcHeadsPerGroup * g;  // this group's first head
-        const uint32_t tcol_l = tl + kColL + hb;   // this thread's row of per-head sums
-        if (e < kTcHeadsPerGroup) ms.mx[g][e] = kNoMax;
-        {
-            float zero[kTcHeadsPerGroup];
-#pragma unroll
-            for (int q = 0; q < kTcHeadsPerGroup; ++q) zero[q] = 0.f;
-            tc_st16(tcol_l, zero);
-            tc_wait_st();
-        }
-        RawTile raw;
-        // tile 0 straight in; tile 1's bytes in flight while the loop starts
-        raw.fetch(a, ms.rows[0][e], g);
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            raw.write(a, V, m, e, g);
+    } else if (warp < 8) {
+        // ------------------------------- producers -------------------------------
+        // After a failed wait the loop still runs to the end, skipping the work, so that every
+        // producer takes the same barriers (the entry-table refills).
+        const int d = threadIdx.x, e = d & (kHalf - 1), cp = d >> 6;
+        RawHalf raw0, raw1;   // half-tiles of even and of odd index
+        raw0.fetch(a, tab[e], cp);
+        if (nh > 1) raw1.fetch(a, tab[kHalf + e], cp);
+        auto step = [&](int t, RawHalf &rw) {
+            const int p = t & 1;
+            if (t >= 2) ok = ok && warp_wait(&ms.v_free[p], ((t >> 1) - 1) & 1, &ms.abort_flag, a.ws, 5);
+            if (ok) rw.write(a, V + p * kVBuf, e, cp);
+            if (cp == 0) {
+                const unsigned int vb = __ballot_sync(0xffffffffu, rw.row != -1);
+                if (lane == 0) reinterpret_cast<volatile uint32_t *>(&ms.vmask[p])[warp] = vb;
+            }
             fence_async_smem();
-            mbar_arrive(&ms.v_ready[m]);
+            mbar_arrive(&ms.v_ready[p]);
+            if (t + 2 < nh) {
+                if ((t + 2) % kTabHalves == 0) {
+                    // the next half-tiles' entry addresses (every producer has fetched from the old ones)
+                    bar_sync(3, kProducers);
+                    fill_table(a, ms, tab, t + 2, d);
+                    bar_sync(3, kProducers);
+                }
+                rw.fetch(a, tab[((t + 2) % kTabHalves) * kHalf + e], cp);
+            }
+        };
+#pragma unroll 1
+        for (int t = 0; t < nh; t += 2) {
+            step(t, raw0);
+            if (t + 1 < nh) step(t + 1, raw1);
         }
-        bool valid_cur = raw.row != -1;
-        if (ntiles > 1) raw.fetch(a, ms.rows[1][e], g);
-        bool ok = warp_wait(&ms.q_ready, 0, &ms.abort_flag, a.ws, 1);
-        ok = group_and(bar_id, ok);   // also orders the maxima's initial values before their first use
-        // After a failed wait the loop still runs to the end, skipping the work, so that every thread
-        // takes the same compute-wide barriers (the entry-table refills); ok is uniform in a group.
-        for (int t = 0; t < ntiles; ++t) {
-            const uint32_t ph = t & 1;
-            ok = group_and(bar_id, ok && warp_wait(&ms.s_full, ph, &ms.abort_flag, a.ws, 6));
+    } else {
+        // ------------------------------- softmax -------------------------------
+        const int sg = (warp - 8) >> 2;         // group: heads 32sg .. 32sg+31
+        const int q = warp & 3;                 // TMEM quarter: lanes 32q .. 32q+31
+        const int gt = threadIdx.x & 127;       // thread within the group
+        const int bar_id = 1 + sg;
+        const int R0 = 16 * q + (lane >> 2);    // half-tile rows of this thread: R0 and R0 + 8
+        const int hc = 2 * (lane & 3);          // head columns: 32sg + 8j + hc, +1 (j = 0..3)
+        float l[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) l[i] = 0.f;
+        ok = warp_wait(&ms.q_ready, 0, &ms.abort_flag, a.ws, 1);
+        for (int t = 0; t < nh; ++t) {
+            const int p = t & 1;
+            const uint32_t ph = (t >> 1) & 1;
+            // v_ready: the producers' valid-row mask of this half-tile; s_full: its scores
+            ok = bar_and(bar_id, 128, ok && warp_wait(&ms.v_ready[p], ph, &ms.abort_flag, a.ws, 9) &&
+                                          warp_wait(&ms.s_full[p], ph, &ms.abort_flag, a.ws, 6));
             if (ok) {
                 tc_fence_after();
-                // scores of this group's 16 heads: the sum of the partial accumulators
-                float z[kTcHeadsPerGroup];
-                load_scores(tl + kColS + hb, valid_cur, zs, z);
+                const uint64_t vm = ms.vmask[p];
+                const bool v0 = (vm >> R0) & 1, v1 = (vm >> (R0 + 8)) & 1;
+                const uint32_t taddr = tmem + ((uint32_t)(32 * q + 16 * p) << 16) + kColS + 32 * sg;
+                float z[16];
+                load_scores(taddr, v0, v1, zs, z);
+                // z[4j + c]: row R0, z[4j + 2 + c]: row R0 + 8; head 32sg + 8j + hc + c
                 bool need = false;
 #pragma unroll
-                for (int q = 0; q < kTcHeadsPerGroup; ++q) need |= z[q] > ms.mx[g][q] + kLazy;
-                if (group_or(bar_id, need)) {
-                    // new maxima: per head one warp max-reduction on order keys, then over the group's warps
+                for (int j = 0; j < 4; ++j)
 #pragma unroll
-                    for (int q = 0; q < kTcHeadsPerGroup; ++q) {
-                        const uint32_t u = __reduce_max_sync(0xffffffffu, order_key(z[q]));
-                        if (lane == 0) ms.red[g][wq][q] = key_to_float(u);
+                    for (int c = 0; c < 2; ++c) {
+                        const float mo = ms.mx[32 * sg + 8 * j + hc + c] + kLazy;
+                        need |= z[4 * j + c] > mo || z[4 * j + 2 + c] > mo;
                     }
-                    group_sync(bar_id);
-                    if (e < kTcHeadsPerGroup) {
-                        const float mt = fmaxf(fmaxf(ms.red[g][0][e], ms.red[g][1][e]), fmaxf(ms.red[g][2][e], ms.red[g][3][e]));
-                        const float mo = ms.mx[g][e];
-                        const float mn = fmaxf(mo, mt);
-                        ms.alpha[g][e] = exp2f(mo - mn);   // 0 while mo is kNoMax
-                        ms.mx[g][e] = mn;
-                    }
-                    group_sync(bar_id);   // new maxima and factors visible; ms.red free again
-                    // this thread's sums, and (after the first tile) this group's head columns of the four
-                    // O^T M-tiles.  PV(t-1) has completed: QK(t) was issued only after every M-tile of
-                    // tile t had been written, each after PV(t-1) had released it (v_free)
-                    {
-                        float lv[kTcHeadsPerGroup];
-                        tc_ld16_sync(tcol_l, lv);
+                if (bar_or(bar_id, 128, need)) {
+                    // new maxima: over this thread's two rows, the warp's 8 row pairs, then the 4 warps
 #pragma unroll
-                        for (int q = 0; q < kTcHeadsPerGroup; ++q) lv[q] *= ms.alpha[g][q];
-                        tc_st16(tcol_l, lv);
-                    }
-                    if (t > 0) {
-#pragma unroll 1
-                        for (int mt = 0; mt < 4; ++mt) {
-                            float o[kTcHeadsPerGroup];
-                            const uint32_t col = kColO + 64 * mt + hb;
-                            tc_ld16_sync(tl + col, o);
+                    for (int j = 0; j < 4; ++j)
 #pragma unroll
-                            for (int q = 0; q < kTcHeadsPerGroup; ++q) o[q] *= ms.alpha[g][q];
-                            tc_st16(tl + col, o);
+                        for (int c = 0; c < 2; ++c) {
+                            float m2 = fmaxf(z[4 * j + c], z[4 * j + 2 + c]);
+                            m2 = fmaxf(m2, __shfl_xor_sync(0xffffffffu, m2, 4));
+                            m2 = fmaxf(m2, __shfl_xor_sync(0xffffffffu, m2, 8));
+                            m2 = fmaxf(m2, __shfl_xor_sync(0xffffffffu, m2, 16));
+                            if (lane < 4) ms.red[sg][q][8 * j + hc + c] = m2;
                         }
+                    bar_sync(bar_id, 128);
+                    if (gt < 32) {
+                        const int h = 32 * sg + gt;
+                        const float mt = fmaxf(fmaxf(ms.red[sg][0][gt], ms.red[sg][1][gt]),
+                                               fmaxf(ms.red[sg][2][gt], ms.red[sg][3][gt]));
+                        const float mo = ms.mx[h];
+                        const float mn = fmaxf(mo, mt);
+                        ms.alpha[h] = exp2f(mo - mn);   // 0 while mo is kNoMax
+                        ms.mx[h] = mn;
                     }
-                    tc_wait_st();
-                    load_scores(tl + kColS + hb, valid_cur, zs, z);   // again, rather than kept live
-                }
-                float lv[kTcHeadsPerGroup];
-                tc_ld16_sync(tcol_l, lv);
-                uint32_t pk[kTcHeadsPerGroup / 2];
+                    bar_sync(bar_id, 128);   // new maxima and factors visible; ms.red free again
 #pragma unroll
-                for (int q = 0; q < kTcHeadsPerGroup; q += 2) {
-                    const float p0 = exp2f(z[q] - ms.mx[g][q] + kPOffset);
-                    const float p1 = exp2f(z[q + 1] - ms.mx[g][q + 1] + kPOffset);
-                    lv[q] += p0;
-                    lv[q + 1] += p1;
-                    pk[q / 2] = pack_f16x2(p0, p1);
+                    for (int j = 0; j < 4; ++j)
+#pragma unroll
+                        for (int c = 0; c < 2; ++c) l[2 * j + c] *= ms.alpha[32 * sg + 8 * j + hc + c];
+                    if (t > 0) {
+                        // this group's head columns of the four O^T M-tiles, once PV(t-1) has completed
+                        const bool pv_ok = warp_wait(&ms.v_free[(t - 1) & 1], ((t - 1) >> 1) & 1, &ms.abort_flag, a.ws, 7);
+                        if (pv_ok) {
+                            tc_fence_after();
+                            const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16);
+#pragma unroll 1
+                            for (int k = 0; k < 8; ++k) {
+                                float o[16];
+                                const uint32_t col = kColO + 64 * (k >> 1) + 32 * sg + 16 * (k & 1);
+                                tc_ld16_sync(tl + col, o);
+#pragma unroll
+                                for (int i = 0; i < 16; ++i) o[i] *= ms.alpha[32 * sg + 16 * (k & 1) + i];
+                                tc_st16(tl + col, o);
+                            }
+                            tc_wait_st();
+                        }
+                        ok = pv_ok;
+                    }
+                    load_scores(taddr, v0, v1, zs, z);   // again, rather than kept live
                 }
-                tc_st16(tcol_l, lv);
-                *reinterpret_cast<uint4 *>(P + swz((uint32_t)e, (uint32_t)(2 * g))) =
-                    make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                *reinterpret_cast<uint4 *>(P + swz((uint32_t)e, (uint32_t)(2 * g + 1))) =
-                    make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                // P^T rows R0, R0 + 8 (entries), this thread's 8 heads: 4-byte pairs
+                uint8_t *Pb = P + p * kPBuf;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int hh = 32 * sg + 8 * j + hc;
+                    const float m0 = ms.mx[hh] - kPOffset, m1 = ms.mx[hh + 1] - kPOffset;
+                    const float p00 = exp2f(z[4 * j] - m0), p01 = exp2f(z[4 * j + 1] - m1);
+                    const float p10 = exp2f(z[4 * j + 2] - m0), p11 = exp2f(z[4 * j + 3] - m1);
+                    l[2 * j] += p00 + p10;
+                    l[2 * j + 1] += p01 + p11;
+                    const uint32_t unit = (uint32_t)(4 * sg + j), off = 4u * (uint32_t)(lane & 3);
+                    *reinterpret_cast<uint32_t *>(Pb + swz((uint32_t)R0, unit) + off) = pack_f16x2(p00, p01);
+                    *reinterpret_cast<uint32_t *>(Pb + swz((uint32_t)(R0 + 8), unit) + off) = pack_f16x2(p10, p11);
+                }
                 fence_async_smem();
-                tc_wait_st();
                 tc_fence_before();
             }
-            mbar_arrive(&ms.p_full);
-            if (t + 1 < ntiles) {
-                // every M-tile of tile t+1 as PV(t) releases it; then the bytes of tile t+2 are
-                // requested, to arrive while tile t+1 is processed
+            mbar_arrive(&ms.p_full[p]);
+        }
+        // softmax denominators: per head, the sum over the group's threads
+        if (bar_and(bar_id, 128, ok)) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int m = release_order(i);
-                    ok = group_and(bar_id, ok && warp_wait(&ms.v_free[m], ph, &ms.abort_flag, a.ws, 5));
-                    if (ok) raw.write(a, V, m, e, g);
-                    fence_async_smem();
-                    mbar_arrive(&ms.v_ready[m]);
-                }
-                valid_cur = raw.row != -1;
-                if (t + 2 < ntiles) {
-                    if ((t + 2) % kTabTiles == 0) {
-                        // the next tiles' entry addresses (every thread has fetched from the old ones)
-                        compute_sync();
-                        fill_table(a, ms, t + 2, ntiles, threadIdx.x);
-                        compute_sync();
-                    }
-                    raw.fetch(a, ms.rows[(t + 2) % kTabTiles][e], g);
+            for (int i = 0; i < 8; ++i) {
+                float v = l[i];
+                v += __shfl_xor_sync(0xffffffffu, v, 4);
+                v += __shfl_xor_sync(0xffffffffu, v, 8);
+                v += __shfl_xor_sync(0xffffffffu, v, 16);
+                l[i] = v;
+            }
+            if (lane < 4) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    ms.red[sg][q][8 * j + hc] = l[2 * j];
+                    ms.red[sg][q][8 * j + hc + 1] = l[2 * j + 1];
                 }
             }
+            bar_sync(bar_id, 128);
+            if (gt < 32) {
+                const int h = 32 * sg + gt;
+                const float lsum = (ms.red[sg][0][gt] + ms.red[sg][1][gt]) + (ms.red[sg][2][gt] + ms.red[sg][3][gt]);
+                float2 *pml = reinterpret_cast<float2 *>(a.part_ml) + ((size_t)b * a.splits + s) * a.H + h0;
+                pml[h] = make_float2((ms.mx[h] - kPOffset) * kLn2, lsum);
+            }
         }
-        // ---- epilogue: this group's share of the split's partial (o, m, l): channels 128g + e of
-        // every head (O^T M-tile g, lane e) and the (m, l) of heads hb .. hb+15
-        float *po = a.part_o + (((size_t)b * a.splits + s) * a.H + h0) * kLatent;
-        float2 *pml = reinterpret_cast<float2 *>(a.part_ml) + ((size_t)b * a.splits + s) * a.H + h0;
-        bool eok = ok && warp_wait(&ms.o_done, 0, &ms.abort_flag, a.ws, 8);
-        eok = group_and(bar_id, eok);
+    }
+    // ---- epilogue: O^T, M-tile w/4, quarter w%4, by every producer and softmax warp
+    if (warp < 16) {
+        const bool eok = bar_and(4, kTcCompute, ok && warp_wait(&ms.o_done, 0, &ms.abort_flag, a.ws, 8));
         if (eok) {
             tc_fence_after();
+            const int m = warp >> 2, qq = warp & 3;
+            float *po = a.part_o + (((size_t)b * a.splits + s) * a.H + h0) * kLatent + 128 * m + 32 * qq + lane;
 #pragma unroll
             for (int hq = 0; hq < kTcHeads; hq += 16) {
                 float o[16];
-                tc_ld16_sync(tmem + ((uint32_t)(wq * 32) << 16) + kColO + 64 * g + hq, o);
+                tc_ld16_sync(tmem + ((uint32_t)(32 * qq) << 16) + kColO + 64 * m + hq, o);
 #pragma unroll
-                for (int q = 0; q < 16; ++q) po[(size_t)(hq + q) * kLatent + 128 * g + e] = o[q];
-            }
-            // softmax denominators: sum of the per-row sums over the group's 128 rows
-            float lv[kTcHeadsPerGroup];
-            tc_ld16_sync(tcol_l, lv);
-#pragma unroll
-            for (int q = 0; q < kTcHeadsPerGroup; ++q) {
-                float v = lv[q];
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                if (lane == 0) ms.red[g][wq][q] = v;
-            }
-            group_sync(bar_id);
-            if (e < kTcHeadsPerGroup) {
-                const float lsum = (ms.red[g][0][e] + ms.red[g][1][e]) + (ms.red[g][2][e] + ms.red[g][3][e]);
-                pml[hb + e] = make_float2((ms.mx[g][e] - kPOffset) * kLn2, lsum);
+                for (int i = 0; i < 16; ++i) po[(size_t)(hq + i) * kLatent] = o[i];
             }
         }
     }
