@@ -7,13 +7,14 @@ A step is one decode step of the whole path over one batch: pack the new token o
 (FP4 + E4M3 key + FP8 window entry), score every block (Full) or the pool (Reindex), exact Top-K,
 sparse attention over the selected FP4 entries plus the FP8 window, and the split combine.  The
 default workload is B=8 sequences of 131,072 tokens, 64 heads, Top-K 2,048 blocks x 8.  Inputs are
-seeded synthetic data resident in HBM; L2 is flushed (256 MB write) before every timed step.
+seeded synthetic data resident in HBM; L2 is flushed (a 256 MB write, then a 256 MB read) before every
+timed step.
 
 Multi-GPU: one process per GPU (torchrun); every rank runs its own batch (data-parallel replicas,
 no collective on the path); the step time is the max over ranks.  Rank 0 prints one JSON line.
 
---impl reference times the CPU oracle (test infrastructure, plain C, one thread) on one sequence
-per step of the same workload.
+--impl reference times the CPU oracle (test infrastructure, plain C, threads over blocks and heads)
+on one sequence per step of the same workload.
 """
 import argparse
 import hashlib
@@ -262,7 +263,15 @@ def run_ours(args, rank, world, local):
     st = workloads.DecodeState(w, device=dev)
     setup_s = time.time() - t0
     plan = make_plan(st)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    # L2 flush before every timed step: write 256 MB, then read another 256 MB, so that no input is
+    # served from L2 and the L2 holds no dirty lines whose write-back would share DRAM with the step
+    flush_w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_r = torch.zeros(256 << 20, dtype=torch.uint8, device=dev)
+
+    def flush_l2():
+        flush_w.zero_()
+        flush_r.sum(dtype=torch.int64)
+
     stream = torch.cuda.current_stream()
 
     def step():
@@ -303,13 +312,13 @@ def run_ours(args, rank, world, local):
     wall0 = time.time()
     if graph is not None:
         for i in range(K):
-            flush.zero_()
+            flush_l2()
             gev[i][0].record(stream)
             graph.replay()
             gev[i][1].record(stream)
     # per-call breakdown: the same step with eager launches and an event around every call
     for i in range(K):
-        flush.zero_()
+        flush_l2()
         for j, (_, _, fn) in enumerate(plan):
             ev[i][j].record(stream)
             fn()
@@ -364,7 +373,7 @@ def run_ours(args, rank, world, local):
     torch.cuda.synchronize()
     e_ms = []
     for i in range(K):
-        flush.zero_()
+        flush_l2()
         a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         e2e_step()
@@ -384,7 +393,7 @@ def run_ours(args, rank, world, local):
             torch.cuda.synchronize()
             g_ms = []
             for i in range(K):
-                flush.zero_()
+                flush_l2()
                 a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 a.record(stream)
                 g2.replay()
@@ -431,7 +440,7 @@ def run_ours(args, rank, world, local):
         "scaling": "weak", "vs_baseline": None, "dtype": "fp4-e2m1/e4m3 KV, f32 indexer, f16 x f16 -> f32 attn",
         "data": "synthetic (seeded; RMSNorm+RoPE latents, N(0,1) keys and queries)",
         "config": {"workload": args.workload, "batch_per_gpu": B, "seq_len": max(w.seq_lens),
-                   "heads": H, "topk_blocks": w.topk, "modes": w.modes, "l2": "flushed (256 MB write) before each step",
+                   "heads": H, "topk_blocks": w.topk, "modes": w.modes, "l2": "flushed before each step (256 MB write, then 256 MB read: no input in L2, no dirty lines)",
                    "parallelism": "dp%d replicas" % world},
         "roofline": roof,
         "step_roofline": {"bytes": step_bytes, "achieved_gbs": round(step_bytes / (max_ms * 1e-3) / 1e9, 1),
@@ -477,6 +486,20 @@ def oracle_step(os_, lat_new, key_new, q, iq, iw, k):
     oracle.attention(q, oracle.default_tau(), os_.codes[pe], os_.scales[pe], os_.swa, os_.swa_scale)
 
 
+def oracle_step_threaded(os_, lat_new, key_new, q, iq, iw, k, threads):
+    """The same decode step on the CPU oracle with its block scores and attention heads spread over
+    threads (the C oracle runs without the GIL)."""
+    import numpy as np
+    import oracle
+    from helpers import attention_threaded, block_scores_threaded
+    oracle.pack_tokens(lat_new, key_new, with_swa=True)
+    S = block_scores_threaded(iq, iw, os_.key8, threads=threads)
+    blocks = oracle.topk(np.arange(S.size, dtype="int32"), S, k)
+    pe = oracle.positions_of_blocks(blocks, os_.L)
+    attention_threaded(q, oracle.default_tau(), os_.codes[pe], os_.scales[pe], os_.swa, os_.swa_scale,
+                       threads=threads)
+
+
 def cpu_cores_info():
     model = ""
     try:
@@ -489,17 +512,24 @@ def cpu_cores_info():
     return model, os.cpu_count()
 
 
-def run_oracle_sample(w, budget_s, max_steps=None, warmup=0):
+def run_oracle_sample(w, budget_s, max_steps=None, warmup=0, threads=1, prepared=None):
     from fp4_compressed_sparse_kv_b200 import workloads
-    os_, lat, key = oracle_sample_setup(w, 0)
+    os_, lat, key = prepared if prepared is not None else oracle_sample_setup(w, 0)
     q, iq, iw = workloads.layer_queries(w, 0)
+
+    def one():
+        if threads == 1:
+            oracle_step(os_, lat, key, q[0], iq[0], iw[0], w.topk)
+        else:
+            oracle_step_threaded(os_, lat, key, q[0], iq[0], iw[0], w.topk, threads)
+
     for _ in range(warmup):
-        oracle_step(os_, lat, key, q[0], iq[0], iw[0], w.topk)
+        one()
     times = []
     t_start = time.time()
     while True:
         t0 = time.time()
-        oracle_step(os_, lat, key, q[0], iq[0], iw[0], w.topk)
+        one()
         times.append(time.time() - t0)
         if max_steps is not None and len(times) >= max_steps:
             break
@@ -513,13 +543,13 @@ def run_reference(args, rank, world):
         return
     from fp4_compressed_sparse_kv_b200 import synth
     w = synth.workload(args.workload)
-    times = run_oracle_sample(w, 0, max_steps=args.steps, warmup=args.warmup)
+    model, ncpu = cpu_cores_info()
+    times = run_oracle_sample(w, 0, max_steps=args.steps, warmup=args.warmup, threads=ncpu)
     s = sum(times)
     value = len(times) / s
-    model, ncpu = cpu_cores_info()
     sample = ("oracle decode step of sequence 0 of %d (context %d, %d heads, Top-K %d): pack of the new "
-              "token, block scores over the whole context, Top-K, attention; one thread" %
-              (w.batch, w.seq_lens[0], w.heads, w.topk))
+              "token, block scores over the whole context, Top-K, attention; block scores and heads over "
+              "%d threads" % (w.batch, w.seq_lens[0], w.heads, w.topk, ncpu))
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": UNIT, "n_gpus": world,
             "steps": len(times), "warmup": args.warmup, "ms_per_step": round(1e3 * s / len(times), 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 attention, f32 indexer",
@@ -528,7 +558,7 @@ def run_reference(args, rank, world):
             "config": {"workload": args.workload, "batch_per_gpu": w.batch, "seq_len": max(w.seq_lens),
                        "heads": w.heads, "topk_blocks": w.topk, "modes": w.modes,
                        "l2": "not applicable (host)", "parallelism": "dp%d replicas" % world},
-            "cpu_baseline": {"value": round(value, 5), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "cpu_baseline": {"value": round(value, 5), "unit": UNIT, "cores": ncpu, "kind": "oracle",
                              "sample": sample, "cpu": model, "host_cpus": ncpu},
             "e2e": {"value": round(value, 5), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -557,12 +587,16 @@ def main():
     if rank == 0 and res is not None:
         line, st = res
         if world == 1 and not args.no_cpu_baseline:
-            times = run_oracle_sample(st.w, args.cpu_seconds)
             model, ncpu = cpu_cores_info()
+            prepared = oracle_sample_setup(st.w, 0)
+            t1 = run_oracle_sample(st.w, args.cpu_seconds / 2, prepared=prepared)
+            tn = run_oracle_sample(st.w, args.cpu_seconds / 2, threads=ncpu, prepared=prepared)
             line["cpu_baseline"] = {
-                "value": round(len(times) / sum(times), 5), "unit": UNIT, "cores": 1, "kind": "oracle",
-                "sample": "%d oracle decode steps of sequence 0 (context %d, %d heads, Top-K %d); one thread"
-                          % (len(times), st.w.seq_lens[0], st.w.heads, st.w.topk),
+                "value": round(len(tn) / sum(tn), 5), "unit": UNIT, "cores": ncpu, "kind": "oracle",
+                "sample": "%d oracle decode steps of sequence 0 (context %d, %d heads, Top-K %d) with block scores "
+                          "and attention heads over %d threads; %d more on one thread"
+                          % (len(tn), st.w.seq_lens[0], st.w.heads, st.w.topk, ncpu, len(t1)),
+                "one_thread": {"value": round(len(t1) / sum(t1), 5), "cores": 1},
                 "cpu": model, "host_cpus": ncpu}
         print(json.dumps(line), flush=True)
     return 0
