@@ -21,6 +21,7 @@ IDX_HEADS = 8
 IDX_DIM = 128
 HEADER_BYTES = 256
 MAX_TOPK = 8192
+MAX_SHARDS = 64
 FULL, REINDEX, REUSE = 0, 1, 2
 
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported configuration", 3: "workspace too small",
@@ -57,7 +58,8 @@ class LayerStepC(ctypes.Structure):
 EXPORTS = ["csa_workspace_bytes", "csa_workspace_init", "csa_kv_pack_fp4", "csa_indexer_full",
            "csa_indexer_reindex", "csa_indexer_block_scores", "csa_topk_blocks", "csa_index_reuse", "csa_sparse_decode_attn", "csa_decode_layer",
            "csa_check_device_error", "csa_status_string", "csa_indexer_full_noalloc",
-           "csa_indexer_screen_bounds", "csa_kv_norm_rope_pack_fp4"]
+           "csa_indexer_screen_bounds", "csa_kv_norm_rope_pack_fp4", "csa_candidates_concat",
+           "csa_shard_blocks", "csa_attn_merge"]
 
 _lib = None
 
@@ -106,6 +108,12 @@ def lib():
     L.csa_indexer_full_noalloc.restype = st
     L.csa_indexer_full_noalloc.argtypes = [ctypes.POINTER(KVLayerC), ctypes.POINTER(BatchC), P, P, i32, P, P,
                                            P, P]
+    L.csa_candidates_concat.restype = st
+    L.csa_candidates_concat.argtypes = [i32, i32, i32, P, P, P, P, P, P, P, P, sz, P]
+    L.csa_shard_blocks.restype = st
+    L.csa_shard_blocks.argtypes = [i32, P, P, i32, P, P, P, P, i32, P, sz, P]
+    L.csa_attn_merge.restype = st
+    L.csa_attn_merge.argtypes = [i32, i32, i32, P, P, P, P, P]
     L.csa_check_device_error.restype = st
     L.csa_check_device_error.argtypes = [P, P, ctypes.POINTER(ctypes.c_int64)]
     L.csa_status_string.restype = ctypes.c_char_p
@@ -319,6 +327,33 @@ def indexer_full_noalloc(layer, batch, iq, iw, k, out_blocks, out_count, dev_sta
                                           _ptr(iw, "iw"), int(k), _ptr(out_blocks, "out_blocks"),
                                           _ptr(out_count, "out_count"), _ptr(dev_status, "dev_status"),
                                           _stream(stream)), "csa_indexer_full_noalloc")
+
+
+def candidates_concat(ids, scores, counts, offsets, out_ids, out_scores, out_count, ws, stream=None):
+    """ids int32 [R, B, cap] (local block ids), scores float32 [R, B, cap], counts / offsets int32
+    [R, B] -> out_ids int32 [B, R * cap] (global ids), out_scores float32 [B, R * cap], out_count [B]."""
+    R, B, cap = (int(x) for x in ids.shape)
+    _check(lib().csa_candidates_concat(R, B, cap, _ptr(ids, "ids"), _ptr(scores, "scores"),
+                                       _ptr(counts, "counts"), _ptr(offsets, "offsets"),
+                                       _ptr(out_ids, "out_ids"), _ptr(out_scores, "out_scores"),
+                                       _ptr(out_count, "out_count"), _ptr(ws, "ws"), ws.numel(),
+                                       _stream(stream)), "csa_candidates_concat")
+
+
+def shard_blocks(blocks, count, lo, hi, out_blocks, out_count, ws, stream=None):
+    """Entries of blocks int32 [B, cap] (count [B]) in [lo[b], hi[b]) minus lo[b], in order."""
+    B, cap = (int(x) for x in blocks.shape)
+    _check(lib().csa_shard_blocks(B, _ptr(blocks, "blocks"), _ptr(count, "count"), cap, _ptr(lo, "lo"),
+                                  _ptr(hi, "hi"), _ptr(out_blocks, "out_blocks"), _ptr(out_count, "out_count"),
+                                  int(out_blocks.shape[1]), _ptr(ws, "ws"), ws.numel(), _stream(stream)),
+           "csa_shard_blocks")
+
+
+def attn_merge(out_parts, lse_parts, out, lse, stream=None):
+    """out_parts float32 [R, B, H, 512], lse_parts float32 [R, B, H] -> out [B, H, 512], lse [B, H]."""
+    R, B, H = (int(x) for x in lse_parts.shape)
+    _check(lib().csa_attn_merge(R, B, H, _ptr(out_parts, "out_parts"), _ptr(lse_parts, "lse_parts"),
+                                _ptr(out, "out"), _ptr(lse, "lse"), _stream(stream)), "csa_attn_merge")
 
 
 def check_device_error(ws, stream=None):

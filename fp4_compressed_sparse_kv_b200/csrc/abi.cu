@@ -161,7 +161,8 @@ csa_status csa_topk_blocks(const csa_batch *batch, const float *scores, int32_t 
     int max_candidates;
     if (pool) {
         if (!pool_count || !aligned16(pool) || !aligned16(pool_count)) return CSA_ERR_INVALID_ARG;
-        if (pool_cap < 1 || pool_cap > CSA_MAX_TOPK || score_stride < pool_cap) return CSA_ERR_INVALID_ARG;
+        if (pool_cap < 1 || pool_cap > CSA_MAX_SHARDS * CSA_MAX_TOPK || score_stride < pool_cap)
+            return CSA_ERR_INVALID_ARG;
         max_candidates = pool_cap;
     } else {
         max_candidates = (batch->max_seq_len + kBlock - 1) / kBlock;

@@ -64,7 +64,9 @@ __device__ __forceinline__ bool seq_view(const AttnArgs &a, int b, SeqView &v)
     }
     v.row = a.swa_row[b];
     v.nF = v.L < kWindow ? v.L : kWindow;
-    if (v.row < 0 || v.row >= a.num_rows) {
+    if (v.row == -1) {
+        v.nF = 0;   // no window segment: a shard that does not hold the sequence's last positions
+    } else if (v.row < 0 || v.row >= a.num_rows) {
         report(a.ws, CSA_ERR_DEVICE_DATA, b);
         v.nF = 0;
     }

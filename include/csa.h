@@ -67,6 +67,7 @@ typedef enum { CSA_FULL = 0, CSA_REINDEX = 1, CSA_REUSE = 2 } csa_layer_mode;
 #define CSA_WINDOW 128
 #define CSA_MAX_SEQ_LEN (1 << 24)
 #define CSA_MAX_TOPK 8192
+#define CSA_MAX_SHARDS 64
 
 /* One KV-producing layer's caches.  All pointers device, caller-owned. */
 typedef struct {
@@ -85,7 +86,8 @@ typedef struct {
     const int32_t *seq_len;      /* device int32 [B], 1 <= seq_len[b] <= max_seq_len */
     const int32_t *block_table;  /* device int32 [B][max_pages]: page id of each 64-token page */
     int32_t max_pages;           /* host: row stride of block_table, >= ceil(max_seq_len / 64) */
-    const int32_t *swa_row;      /* device int32 [B]: the sequence's row of the SWA ring */
+    const int32_t *swa_row;      /* device int32 [B]: the sequence's row of the SWA ring; -1 = no window
+                                    segment (attention of a context shard without the last positions) */
     int32_t max_seq_len;         /* host: upper bound of seq_len[], sizes grids and workspace */
 } csa_batch;
 
@@ -206,7 +208,8 @@ csa_status csa_indexer_block_scores(const csa_kv_layer *layer, const csa_batch *
 /*
  * Step 3 alone -- exact Top-k of block scores from csa_indexer_block_scores (same pool arguments):
  * larger score first, then lower block id; the min(k, n) chosen block ids are written ascending.
- * Bit-for-bit defined.  ws needs CSA_WORKSPACE_HEADER_BYTES.
+ * In pool mode pool_cap may be up to CSA_MAX_SHARDS * CSA_MAX_TOPK (a concatenation of candidate
+ * lists, csa_candidates_concat).  Bit-for-bit defined.  ws needs CSA_WORKSPACE_HEADER_BYTES.
  */
 csa_status csa_topk_blocks(const csa_batch *batch, const float *scores, int32_t score_stride,
                            const int32_t *pool, const int32_t *pool_count, int32_t pool_cap,
@@ -297,6 +300,49 @@ csa_status csa_indexer_full_noalloc(const csa_kv_layer *layer, const csa_batch *
                                     const uint16_t *iq, const float *iw, int32_t k,
                                     int32_t *out_blocks, int32_t *out_count, int32_t *dev_status,
                                     void *stream);
+
+/*
+ * Context-parallel decode of a long sequence: its positions split into R contiguous slices, rank r
+ * holding slice [s_r, e_r) (page-aligned, ascending in r) in its own caches, with a batch view of the
+ * slice (seq_len = e_r - s_r, swa_row = -1 except on the rank holding the last positions).  Each rank
+ * runs csa_indexer_full(k) on its slice and csa_indexer_block_scores on the chosen blocks (their
+ * exact scores); the ranks exchange those lists; the Top-k of the concatenated list (csa_topk_blocks
+ * in pool mode, over the whole sequence's batch view) is the Full layer's exact Top-k ([rebasdaily]
+ * 同一份笔记，多层一起用: the full-range scan, here sharded by position), since every block of the
+ * global Top-k is in its own slice's Top-k.  Each rank attends over its part of that set
+ * (csa_shard_blocks, then csa_sparse_decode_attn on its slice), and the ranks' (out, lse) merge
+ * exactly (csa_attn_merge).  The exchanges themselves (all-gathers) are the caller's, e.g. NCCL.
+ *
+ * csa_candidates_concat -- per sequence b, the R lists ids[r][b][0 .. counts[r][b]) (local block
+ *   ids, ascending) plus offsets[r][b] (the slice's first block) with their scores, into one list
+ *   out_ids[b][0 .. out_count[b]) of global ids (ascending when the slices are) and out_scores.
+ *     ids int32 [R][B][cap], scores float [R][B][cap], counts int32 [R][B] (<= cap), offsets int32 [R][B]
+ *     out_ids int32 [B][R * cap], out_scores float [B][R * cap], out_count int32 [B]
+ *   1 <= R <= CSA_MAX_SHARDS.  ws needs CSA_WORKSPACE_HEADER_BYTES (a count out of range is reported).
+ */
+csa_status csa_candidates_concat(int32_t R, int32_t B, int32_t cap, const int32_t *ids, const float *scores,
+                                 const int32_t *counts, const int32_t *offsets, int32_t *out_ids,
+                                 float *out_scores, int32_t *out_count, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * csa_shard_blocks -- per sequence b, the entries v of blocks[b][0 .. count[b]) with
+ * lo[b] <= v < hi[b], as v - lo[b], in their order, into out_blocks[b][0 .. out_count[b]).
+ *     blocks int32 [B][cap], count int32 [B], lo, hi int32 [B], out_blocks int32 [B][out_cap]
+ *   More than out_cap entries in range are reported and cut at out_cap.
+ */
+csa_status csa_shard_blocks(int32_t B, const int32_t *blocks, const int32_t *count, int32_t cap,
+                            const int32_t *lo, const int32_t *hi, int32_t *out_blocks, int32_t *out_count,
+                            int32_t out_cap, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * csa_attn_merge -- attention over the union of R disjoint entry sets from the attention over each:
+ * lse = log sum_r e^{lse_r}, out = sum_r e^{lse_r - lse} out_r (a set with lse_r = -inf, i.e. no
+ * entry, takes no part; if every set is empty, out = 0 and lse = -inf).
+ *     out_parts float [R][B][H][512], lse_parts float [R][B][H]; out float [B][H][512], lse float [B][H]
+ *   1 <= R <= CSA_MAX_SHARDS, H in {16, 32, 64, 128}.
+ */
+csa_status csa_attn_merge(int32_t R, int32_t B, int32_t H, const float *out_parts, const float *lse_parts,
+                          float *out, float *lse, void *stream);
 
 /* Synchronise `stream`, read and clear the workspace status word.  Returns CSA_OK,
  * CSA_ERR_DEVICE_DATA or CSA_ERR_TIMEOUT; *detail (host, may be NULL) receives the first
