@@ -42,6 +42,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time eager launches only")
+    ap.add_argument("--no-tier", action="store_true", help="skip the persistent-tier copy measurement")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU baseline sample budget")
     return ap.parse_args()
 
@@ -244,6 +245,58 @@ def attn_flops(st):
     return total
 
 
+def measure_kv_tier(st, dev, flush_l2, hbm_gbs, reps=3):
+    """Export and import of every sequence's persistent record (FP4 codes, scales, indexer keys) of
+    the first KV layer, to and from HBM and pinned host memory: one csa_kv_export / csa_kv_import per
+    sequence, timed with CUDA events over the whole batch after an L2 flush."""
+    import torch
+
+    from fp4_compressed_sparse_kv_b200 import csa
+    w, lay = st.w, st.layers[0]
+    lens = [int(x) for x in w.seq_lens]
+    sizes = [csa.kv_record_bytes(n) for n in lens]
+    offs = [sum(sizes[:b]) for b in range(len(sizes))]
+    total = sum(sizes)
+    bufs = {"hbm": torch.empty((total,), dtype=torch.uint8, device=dev),
+            "host": torch.empty((total,), dtype=torch.uint8).pin_memory()}
+    rows = [st.batch.block_table[b].clone() for b in range(len(lens))]   # 16-byte aligned rows
+    ws = csa.workspace(1, 16, 64, 8, device=dev)
+    stream = torch.cuda.current_stream()
+    out = {"record_bytes": total, "sequences": len(lens), "bytes_per_token": 416}
+
+    def run(kind, where):
+        fn = csa.kv_export if kind == "export" else csa.kv_import
+        buf = bufs[where]
+        for b, n in enumerate(lens):
+            fn(lay, rows[b], n, buf[offs[b]:offs[b] + sizes[b]], ws)
+
+    for kind in ("export", "import"):
+        for where in ("hbm", "host"):
+            run(kind, where)
+            torch.cuda.synchronize()
+            ms = []
+            for _ in range(reps):
+                flush_l2()
+                a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                run(kind, where)
+                b_.record(stream)
+                b_.synchronize()
+                ms.append(a.elapsed_time(b_))
+            t = sum(ms) / reps
+            # HBM to HBM moves every byte twice through DRAM (read + write); to or from the host each
+            # byte crosses the host link once and DRAM once
+            moved = 2 * total if where == "hbm" else total
+            rec = {"ms": round(t, 4), "gbs": round(moved / (t * 1e-3) / 1e9, 1)}
+            if where == "hbm":
+                rec["hbm_frac"] = round(moved / (t * 1e-3) / 1e9 / hbm_gbs, 4)
+            out["%s_%s" % (kind, where)] = rec
+    st.check()
+    if csa.check_device_error(ws)[0] != 0:
+        raise RuntimeError("persistent-tier copy reported a device-data error")
+    return out
+
+
 def run_ours(args, rank, world, local):
     import numpy as np
     import torch
@@ -408,6 +461,7 @@ def run_ours(args, rank, world, local):
         return None
 
     peaks = measured_peaks()
+    tier = None if args.no_tier else measure_kv_tier(st, dev, flush_l2, peaks["hbm_gbs"])
     dominant = max(call_ms, key=call_ms.get)
     kernels = {}
     for n in call_ms:
@@ -453,6 +507,7 @@ def run_ours(args, rank, world, local):
                 "timing": ("CUDA-graph replay of copies in + public calls + copies out, host synchronised each step"
                            if e2e_graph else "eager public calls with the copies, host synchronised each step"),
                 "eager": {"value": round(world * B / (e2e_eager_ms * 1e-3), 2), "ms_per_step": round(e2e_eager_ms, 5)}},
+        "kv_tier": tier,
         "gpu_launches": (2 if graph is not None else 1) * K * sum(k for _, k, _ in plan),
         "timing": ("CUDA-graph replay of the step (headline); per-kernel figures from eager launches "
                    "with an event around every call, eager step %.5f ms" % eager_ms) if graph is not None

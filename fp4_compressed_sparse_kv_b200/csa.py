@@ -59,7 +59,7 @@ EXPORTS = ["csa_workspace_bytes", "csa_workspace_init", "csa_kv_pack_fp4", "csa_
            "csa_indexer_reindex", "csa_indexer_block_scores", "csa_topk_blocks", "csa_index_reuse", "csa_sparse_decode_attn", "csa_decode_layer",
            "csa_check_device_error", "csa_status_string", "csa_indexer_full_noalloc",
            "csa_indexer_screen_bounds", "csa_kv_norm_rope_pack_fp4", "csa_candidates_concat",
-           "csa_shard_blocks", "csa_attn_merge"]
+           "csa_shard_blocks", "csa_attn_merge", "csa_kv_record_bytes", "csa_kv_export", "csa_kv_import"]
 
 _lib = None
 
@@ -114,6 +114,12 @@ def lib():
     L.csa_shard_blocks.argtypes = [i32, P, P, i32, P, P, P, P, i32, P, sz, P]
     L.csa_attn_merge.restype = st
     L.csa_attn_merge.argtypes = [i32, i32, i32, P, P, P, P, P]
+    L.csa_kv_record_bytes.restype = sz
+    L.csa_kv_record_bytes.argtypes = [i32]
+    L.csa_kv_export.restype = st
+    L.csa_kv_export.argtypes = [ctypes.POINTER(KVLayerC), P, i32, P, P, sz, P]
+    L.csa_kv_import.restype = st
+    L.csa_kv_import.argtypes = [ctypes.POINTER(KVLayerC), P, i32, P, P, sz, P]
     L.csa_check_device_error.restype = st
     L.csa_check_device_error.argtypes = [P, P, ctypes.POINTER(ctypes.c_int64)]
     L.csa_status_string.restype = ctypes.c_char_p
@@ -134,6 +140,17 @@ def _ptr(t, name):
         raise TypeError("%s must be a torch tensor" % name)
     if not t.is_cuda:
         raise ValueError("%s must be a CUDA tensor (the library has no CPU path)" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    return t.data_ptr()
+
+
+def _buf_ptr(t, name):
+    """A device tensor, or a page-locked host tensor (the kernel reads or writes it over the bus)."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch tensor" % name)
+    if not (t.is_cuda or t.is_pinned()):
+        raise ValueError("%s must be a CUDA tensor or a pinned host tensor" % name)
     if not t.is_contiguous():
         raise ValueError("%s must be contiguous" % name)
     return t.data_ptr()
@@ -354,6 +371,35 @@ def attn_merge(out_parts, lse_parts, out, lse, stream=None):
     R, B, H = (int(x) for x in lse_parts.shape)
     _check(lib().csa_attn_merge(R, B, H, _ptr(out_parts, "out_parts"), _ptr(lse_parts, "lse_parts"),
                                 _ptr(out, "out"), _ptr(lse, "lse"), _stream(stream)), "csa_attn_merge")
+
+
+def kv_record_bytes(n):
+    """Bytes of the persistent record of an n-token sequence: 26,624 per 64-token page."""
+    return int(lib().csa_kv_record_bytes(int(n)))
+
+
+def _record_args(layer, block_table, n, buf, name):
+    if buf.dtype != torch.uint8 or buf.numel() < kv_record_bytes(n):
+        raise ValueError("%s must be a uint8 tensor of at least kv_record_bytes(n) bytes" % name)
+    if block_table.dtype != torch.int32 or block_table.numel() < (int(n) + PAGE - 1) // PAGE:
+        raise ValueError("block_table must be int32 with one entry per page of the sequence")
+    return layer.c(), _ptr(block_table, "block_table"), _buf_ptr(buf, name)
+
+
+def kv_export(layer, block_table, n, dst, ws, stream=None):
+    """Copy the persistent record (FP4 codes, scales, indexer keys; no window) of the n-token sequence
+    whose pages are block_table[0 .. ceil(n/64)) into dst (device, or pinned host)."""
+    lc, bt, d = _record_args(layer, block_table, n, dst, "dst")
+    _check(lib().csa_kv_export(ctypes.byref(lc), bt, int(n), d, _ptr(ws, "ws"), ws.numel(), _stream(stream)),
+           "csa_kv_export")
+
+
+def kv_import(layer, block_table, n, src, ws, stream=None):
+    """Write a persistent record back into the pages block_table[0 .. ceil(n/64)).  The window is
+    restored afterwards by replaying the last min(n, 128) tokens through kv_pack_fp4."""
+    lc, bt, s = _record_args(layer, block_table, n, src, "src")
+    _check(lib().csa_kv_import(ctypes.byref(lc), bt, int(n), s, _ptr(ws, "ws"), ws.numel(), _stream(stream)),
+           "csa_kv_import")
 
 
 def check_device_error(ws, stream=None):

@@ -344,6 +344,34 @@ csa_status csa_shard_blocks(int32_t B, const int32_t *blocks, const int32_t *cou
 csa_status csa_attn_merge(int32_t R, int32_t B, int32_t H, const float *out_parts, const float *lse_parts,
                           float *out, float *lse, void *stream);
 
+/*
+ * Persistent KV tier ([yomxxx] 三 "让 KV 不必一直待在 HBM 里": the global KV stays in HBM, the
+ * persistent KV goes to SSD or host memory and is fetched back when needed; [rebasdaily]
+ * 先让长输入少走一半路, SWA Bounded Replay: the sliding-window state is not stored, the most recent
+ * tokens are replayed to restore it).  A sequence's persistent record holds its FP4 codes, E4M3
+ * scales and E4M3 indexer keys and nothing of the window: one 26,624-byte record per 64-token page
+ * (416 B per token), laid out
+ *     codes [64][256] | scales [64][32] | keys [64][128]
+ * for page i of the sequence (block_table[i]), i = 0 .. ceil(n / 64) - 1, back to back.  Rows of the
+ * last page past n are copied as they are.  To restore a sequence: csa_kv_import into any pages,
+ * then csa_kv_pack_fp4 of its last min(n, 128) tokens with their window slots (the replay; it writes
+ * those tokens' FP4 and key bytes again, identically, and the window).
+ *
+ * csa_kv_record_bytes -- ceil(n / 64) * 26,624 (0 for n < 0).
+ * csa_kv_export / csa_kv_import -- copy the record out of / into the pages block_table[0 ..
+ *   ceil(n / 64)) (device int32) of `layer`.  dst / src is device memory or page-locked host memory
+ *   (cudaHostAlloc, cudaMallocHost, or cudaHostRegister'd); any other host pointer returns
+ *   CSA_ERR_INVALID_ARG before any launch.  The copy runs as one kernel on `stream`: a host buffer is
+ *   written or read over the bus by the kernel itself.  A page id out of [0, num_pages) is reported
+ *   and its record skipped.  0 <= n <= CSA_MAX_SEQ_LEN; n = 0 is a no-op.  ws needs
+ *   CSA_WORKSPACE_HEADER_BYTES.  Bit-for-bit.
+ */
+size_t csa_kv_record_bytes(int32_t n);
+csa_status csa_kv_export(const csa_kv_layer *layer, const int32_t *block_table, int32_t n, uint8_t *dst,
+                         void *ws, size_t ws_bytes, void *stream);
+csa_status csa_kv_import(const csa_kv_layer *layer, const int32_t *block_table, int32_t n, const uint8_t *src,
+                         void *ws, size_t ws_bytes, void *stream);
+
 /* Synchronise `stream`, read and clear the workspace status word.  Returns CSA_OK,
  * CSA_ERR_DEVICE_DATA or CSA_ERR_TIMEOUT; *detail (host, may be NULL) receives the first
  * offending index recorded. */

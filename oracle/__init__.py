@@ -279,6 +279,18 @@ def attend(layer, block_table_row, swa_row, L, q, tau, blocks, W=WINDOW):
                      layer["swa"][swa_row, slots], layer["swa_scale"][swa_row, slots])
 
 
+def persistent_record(layer, block_table_row, n):
+    """A sequence's persistent record: for each of its ceil(n/64) pages, in order, the page's codes
+    [64][256], scales [64][32] and indexer keys [64][128] back to back; no window entry ([yomxxx] 三:
+    the persistent KV tier in host memory or on SSD; [rebasdaily] 先让长输入少走一半路, SWA Bounded
+    Replay: the window is restored by replaying the last tokens, not stored)."""
+    pages = np.asarray(block_table_row, np.int64)[:(n + PAGE - 1) // PAGE]
+    parts = []
+    for p in pages:
+        parts += [layer["codes"][p].reshape(-1), layer["scales"][p].reshape(-1), layer["keys"][p].reshape(-1)]
+    return np.concatenate(parts) if parts else np.zeros((0,), np.uint8)
+
+
 def default_tau():
     """Softmax temperature 1/sqrt(512) (the pages give none)."""
     return 1.0 / math.sqrt(LATENT)

@@ -111,3 +111,15 @@ def test_binding_refuses_host_tensors():
     from fp4_compressed_sparse_kv_b200 import csa
     with pytest.raises(ValueError):
         csa._ptr(torch.zeros(4), "x")
+
+
+def test_persistent_record_sizes_and_host_checks(lib):
+    import ctypes as C
+    for n, want in [(0, 0), (1, 26624), (64, 26624), (65, 53248), (1 << 20, 16384 * 26624), (-1, 0)]:
+        assert lib.csa_kv_record_bytes(n) == want
+    ws = (C.c_uint8 * 272)()
+    wsp = (C.addressof(ws) + 15) // 16 * 16
+    # n = 0 is a no-op; a null layer or a negative n is refused before anything reaches the device
+    assert lib.csa_kv_export(None, None, 0, None, None, 0, None) == 0
+    assert lib.csa_kv_export(None, C.c_void_p(wsp), 64, C.c_void_p(wsp), C.c_void_p(wsp), 256, None) == 1
+    assert lib.csa_kv_import(None, C.c_void_p(wsp), -5, C.c_void_p(wsp), C.c_void_p(wsp), 256, None) == 1

@@ -205,3 +205,63 @@ def test_large_k_over_interleaved_magnitudes(layout):
     got = full_select(layer, batch, iq, iw, k)
     exact = oracle.block_scores(iq[0], iw[0], keys[0])
     assert got[0].tolist() == oracle.topk(np.arange(n, dtype=np.int32), exact, k).tolist()
+
+
+def cancelling_keys(rng, n, jr=(1, 17), M_choices=(448.0, 240.0, 96.0, 26.0)):
+    """Every position, in each 32-channel slice (one K=32 tensor-core step): 15 channels +M, 15
+    channels -M (M per position and slice), at random places, and two residue channels of magnitude
+    M 2^-j, j uniform in jr, random signs.  With a query constant over the slice, the large
+    products cancel exactly and leave a residue from 2^-1 down to 2^-17 of the largest product."""
+    keys = np.zeros((n, 128), np.float32)
+    for s in range(4):
+        M = rng.choice(np.array(M_choices, np.float32), size=n)
+        sl = np.zeros((n, 32), np.float32)
+        sl[:, :15] = M[:, None]
+        sl[:, 15:30] = -M[:, None]
+        j = rng.uniform(jr[0], jr[1], size=(n, 2))
+        sl[:, 30:] = (M[:, None] * np.exp2(-j) * rng.choice([-1.0, 1.0], size=(n, 2))).astype(np.float32)
+        perm = np.argsort(rng.random((n, 32)), axis=1)
+        keys[:, 32 * s:32 * (s + 1)] = np.take_along_axis(sl, perm, axis=1)
+    return oracle.e4m3_encode(keys)
+
+
+def test_bounds_bracket_exact_scores_under_slice_cancellation():
+    """The accumulation constant of the bound (the tensor core's fp32 sum of one K=32 step errs by at
+    most 2^-14 of the sum of its product magnitudes) under the worst case for it: in every slice the
+    large products cancel exactly and only residues far below them remain.  Head h reads only slice
+    h mod 4 (its query is a constant there, zero elsewhere), so its bound is about 2^-14 x 32 |c| M and
+    the residues land on both sides of it; a tensor core that dropped or truncated the residues by more
+    than the constant would push exact scores out of their brackets.  The screened Top-K must also
+    equal the oracle's."""
+    rng = np.random.default_rng(21)
+    lens = [1, 100, 1000, 4099]
+    jr = [(1, 17), (6, 12), (9, 17), (1, 17)]
+    keys = [cancelling_keys(rng, L, j) for L, j in zip(lens, jr)]
+    B = len(lens)
+    c = synth.bf16_to_f32(synth.bf16_bits(rng.uniform(0.5, 3.0, size=(B, 8)).astype(np.float32)))
+    c *= rng.choice([-1.0, 1.0], size=(B, 8)).astype(np.float32)
+    q = np.zeros((B, 8, 128), np.float32)
+    for h in range(8):
+        s = h % 4
+        q[:, h, 32 * s:32 * (s + 1)] = c[:, h, None]
+    iq = synth.bf16_bits(q)
+    iw = rng.random((B, 8)).astype(np.float32)
+    layer, batch = gpu_layer(keys, 9)
+    lo, hi = screen(layer, batch, iq, iw)
+    below = above = 0
+    for b, L in enumerate(lens):
+        nb = (L + 7) // 8
+        exact = oracle.block_scores(iq[b], iw[b], keys[b])
+        l, h = lo[b, :nb], hi[b, :nb]
+        bad = np.nonzero(~((l <= exact) & (exact <= h)))[0]
+        assert bad.size == 0, "seq %d block %d: %r not in [%r, %r]" % (b, bad[0], exact[bad[0]], l[bad[0]], h[bad[0]])
+        half = (h - l) / 2
+        below += int((exact < half).sum())
+        above += int((exact > 4 * half).sum())
+    # the residues straddle the bound: some blocks score below the bracket's half-width, some far above
+    assert below > 0 and above > 0, (below, above)
+    k = 40
+    got = full_select(layer, batch, iq, iw, k)
+    for b, L in enumerate(lens):
+        exact = oracle.block_scores(iq[b], iw[b], keys[b])
+        assert got[b].tolist() == oracle.topk(np.arange(len(exact), dtype=np.int32), exact, k).tolist()
