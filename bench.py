@@ -177,9 +177,8 @@ def make_plan(st):
         lay = st.layers[f]
         if m == csa.FULL:
             plan.append(("kv_pack_fp4", 1, lambda f=f: st.pack_new_tokens(f)))
-            # query terms, screen, two classification passes, exact re-score, finalize (one launch when
-            # every block is selected)
-            n_full = 1 if (st.max_seq_len + 7) // 8 <= st.layer_k[l] else 6
+            # query terms, screen, selection (one launch when every block is selected)
+            n_full = 1 if (st.max_seq_len + 7) // 8 <= st.layer_k[l] else 3
             plan.append(("indexer_full", n_full,
                          lambda l=l, lay=lay: csa.indexer_full(lay, st.batch, st.iq[l], st.iw[l], st.layer_k[l],
                                                                st.blocks[l], st.count[l], st.ws)))

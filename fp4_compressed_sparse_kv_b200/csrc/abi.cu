@@ -22,20 +22,15 @@ cudaError_t launch_block_scores_full_or_pool(const uint8_t *keys, int num_pages,
                                              const uint16_t *iq, const float *iw, const int32_t *pool,
                                              const int32_t *pool_count, int pool_cap, float *scores,
                                              int score_stride, void *ws, cudaStream_t st);
-cudaError_t launch_block_scores_list(const uint8_t *keys, int num_pages, const csa_batch &bt, const uint16_t *iq,
-                                     const float *iw, const uint2 *list, const int32_t *list_count, float *scores,
-                                     int score_stride, void *ws, cudaStream_t st);
 bool screen_supported(int num_pages);
 cudaError_t launch_screen_bounds(const uint8_t *keys, int num_pages, const csa_batch &bt, const uint16_t *iq,
-                                 const float *iw, uint8_t *qt, void *qm, int32_t *list_count, uint32_t *hist,
-                                 uint32_t *hist2, void *words, float *lo, float *hi, int stride, void *ws,
-                                 cudaStream_t st);
-cudaError_t launch_classify(const float *lo, const float *hi, int stride, const csa_batch &bt, int k,
-                            const uint32_t *hist, uint32_t *hist2, void *words, uint8_t *status, int sstride,
-                            int32_t *uslice, uint2 *list, int32_t *list_count, void *ws, cudaStream_t st);
-cudaError_t launch_finalize(const float *scores, int score_stride, const csa_batch &bt, uint8_t *status,
-                            int sstride, const int32_t *uslice, const void *words, int stride, int k,
-                            int32_t *out_blocks, int32_t *out_count, void *ws, cudaStream_t st);
+                                 const float *iw, uint8_t *qt, void *qm, uint32_t *hist, uint32_t *hist2, float *lo,
+                                 float *hi, int stride, void *ws, cudaStream_t st);
+cudaError_t launch_select(const float *lo, const float *hi, int lstride, const csa_batch &bt, int k,
+                          const uint32_t *hist, uint32_t *hist2, uint8_t *status, int sstride, int32_t *uslice,
+                          uint32_t *okeys, int ustride, uint32_t *takes, const uint8_t *keys, int num_pages,
+                          const uint16_t *iq, const float *iw, int32_t *out_blocks, int32_t *out_count, void *ws,
+                          cudaStream_t st);
 cudaError_t launch_attn_tc(const AttnArgs &a, cudaStream_t st);
 bool attn_tc_supported(int H);
 bool attn_tc_layer_ok(int num_pages, int num_rows);
@@ -214,23 +209,16 @@ csa_status csa_indexer_full(const csa_kv_layer *layer, const csa_batch *batch, c
     float *hi = reinterpret_cast<float *>(base + w.hi);
     uint32_t *hist = reinterpret_cast<uint32_t *>(base + w.hist);
     uint32_t *hist2 = reinterpret_cast<uint32_t *>(base + w.hist2);
-    void *words = base + w.topk;
     uint8_t *status = reinterpret_cast<uint8_t *>(base + w.status);
     int32_t *uslice = reinterpret_cast<int32_t *>(base + w.uslice);
-    uint2 *list = reinterpret_cast<uint2 *>(base + w.list);
-    int32_t *list_count = reinterpret_cast<int32_t *>(base + w.list_count);
+    const int lstride = (int)w.lstride;
     cudaError_t e = launch_screen_bounds(layer->keys, layer->num_pages, *batch, iq, iw,
-                                         reinterpret_cast<uint8_t *>(base + w.qt), base + w.qm, list_count, hist,
-                                         hist2, words, lo, hi, nb, ws, st);
-    if (e == cudaSuccess)
-        e = launch_classify(lo, hi, nb, *batch, k, hist, hist2, words, status, (int)w.status_stride, uslice, list,
-                            list_count, ws, st);
-    if (e == cudaSuccess)
-        e = launch_block_scores_list(layer->keys, layer->num_pages, *batch, iq, iw, list, list_count, scores,
-                                     (int)w.score_cap, ws, st);
-    if (e == cudaSuccess)
-        e = launch_finalize(scores, (int)w.score_cap, *batch, status, (int)w.status_stride, uslice, words, nb, k,
-                            out_blocks, out_count, ws, st);
+                                         reinterpret_cast<uint8_t *>(base + w.qt), base + w.qm, hist, hist2, lo, hi,
+                                         lstride, ws, st);
+    if (e == cudaSuccess)   // the score region (B x score_cap >= B x nb words) keeps the overflow keys
+        e = launch_select(lo, hi, lstride, *batch, k, hist, hist2, status, (int)w.status_stride, uslice,
+                          reinterpret_cast<uint32_t *>(scores), nb, reinterpret_cast<uint32_t *>(base + w.topk),
+                          layer->keys, layer->num_pages, iq, iw, out_blocks, out_count, ws, st);
     return cuda_status(e);
 }
 
@@ -249,9 +237,8 @@ csa_status csa_indexer_screen_bounds(const csa_kv_layer *layer, const csa_batch 
     char *base = (char *)ws;
     return cuda_status(launch_screen_bounds(layer->keys, layer->num_pages, *batch, iq, iw,
                                             reinterpret_cast<uint8_t *>(base + w.qt), base + w.qm,
-                                            reinterpret_cast<int32_t *>(base + w.list_count),
-                                            reinterpret_cast<uint32_t *>(base + w.hist), nullptr, nullptr, lower, upper,
-                                            stride, ws, (cudaStream_t)stream));
+                                            reinterpret_cast<uint32_t *>(base + w.hist), nullptr, lower, upper, stride,
+                                            ws, (cudaStream_t)stream));
 }
 
 csa_status csa_indexer_reindex(const csa_kv_layer *layer, const csa_batch *batch, const uint16_t *iq,

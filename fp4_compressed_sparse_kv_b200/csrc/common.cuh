@@ -32,18 +32,17 @@ constexpr int kAttnUnit = 8;                // entries per attention work unit (
 constexpr int kWindowUnits = kWindow / kAttnUnit;
 
 struct WsLayout {
-    size_t scores = 0;       // float [B][score_cap]
+    size_t scores = 0;       // float [B][score_cap] (the Full selection keeps uint32 score keys here)
     size_t score_cap = 0;
-    size_t topk = 0;         // uint32 [B][topk_words] per-sequence select state
+    size_t topk = 0;         // uint32 [B][topk_words] per-sequence select state (words, counts)
     size_t nb = 0;           // blocks of the longest sequence
-    size_t lo = 0, hi = 0;   // float [B][nb] screening bounds of every block
+    size_t lo = 0, hi = 0;   // float [B][lstride] screening bounds of every block
+    size_t lstride = 0;      // nb rounded up to 4 (16-byte rows)
     size_t qt = 0;           // uint8 [B][kQtBytes] query-term operand images
     size_t qm = 0;           // [B][kQmBytes] per-sequence screening constants
-    size_t status = 0;       // uint8 [B][status_stride] class of every block (out, sure, uncertain, ...)
+    size_t status = 0;       // uint8 [B][status_stride] class of every block (out, sure, uncertain, chosen)
     size_t status_stride = 0;   // nb rounded up to 16
-    size_t uslice = 0;       // int32 [B][nb] each sequence's uncertain blocks, any order
-    size_t list = 0;         // uint2 [B * nb] re-scoring work list (b, block)
-    size_t list_count = 0;   // int32 entries in the list
+    size_t uslice = 0;       // int32 [B][nb] uncertain blocks beyond the selection's shared-memory lists
     size_t hist = 0;         // uint32 [B][kHistBins] histogram of the blocks' lower-bound keys
     size_t hist2 = 0;        // uint32 [B][kHistBins] second level, inside the threshold bin
     size_t screen_end = 0;   // end of the indexer's regions
@@ -86,10 +85,11 @@ inline WsLayout ws_layout(int B, int H, int max_seq_len, int cap, int units_per_
     w.topk = o;
     o = align_up(o + (size_t)B * kTopkWords * 4, 256);
     w.nb = nb;
+    w.lstride = align_up(nb, 4);
     w.lo = o;
-    o = align_up(o + (size_t)B * nb * 4, 256);
+    o = align_up(o + (size_t)B * w.lstride * 4, 256);
     w.hi = o;
-    o = align_up(o + (size_t)B * nb * 4, 256);
+    o = align_up(o + (size_t)B * w.lstride * 4, 256);
     w.qt = o;
     o = align_up(o + (size_t)B * kQtBytes, 1024);
     w.qm = o;
@@ -99,10 +99,6 @@ inline WsLayout ws_layout(int B, int H, int max_seq_len, int cap, int units_per_
     o = align_up(o + (size_t)B * w.status_stride, 256);
     w.uslice = o;
     o = align_up(o + (size_t)B * nb * 4, 256);
-    w.list = o;
-    o = align_up(o + (size_t)B * nb * 8, 256);
-    w.list_count = o;
-    o = align_up(o + 4, 256);
     w.hist = o;
     o = align_up(o + (size_t)B * kHistBins * 4, 256);
     w.hist2 = o;

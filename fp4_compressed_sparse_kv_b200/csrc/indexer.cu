@@ -11,23 +11,19 @@
 #include "convert.cuh"
 #include "pipeline.cuh"
 #include "radix.cuh"
+#include "score.cuh"
 
 namespace csa {
 
 // ------------------------------------------------------------------------------------------------
 // Block scoring.  Persistent CTAs of 8 warps; a work item is 8 consecutive "virtual" blocks of one
 // sequence (in Full mode virtual block v is block v, so an item is one 64-token page; in Reindex
-// mode it is pool[b][v]) and warp w always takes virtual block w of each item.  In list mode an item
-// is 8 consecutive entries (b, block) of a device-built work list, warp w taking entry w, and the
-// score goes to scores[b][block]; the list holds only real work.  Every warp runs its
+// mode it is pool[b][v]) and warp w always takes virtual block w of each item.  Every warp runs its
 // own pipeline: lane 0 resolves the block's page a few items ahead and bulk-copies its 1 KB of keys
 // into the warp's shared-memory ring; no warp ever waits for another.
 //
-// Lane (g, j) = (lane/8, lane%8) holds dims 16j..16j+15 of all 8 query heads in registers and takes
-// key g of each group of 4.  Lane j keeps head s^j in register slot s, so the 3-step xor
-// reduce-scatter (distances 4, 2, 1) needs no selects and leaves head j in lane j, having formed
-// exactly ((p0+p4)+(p2+p6)) + ((p1+p5)+(p3+p7)) up to the commutativity of each addition.  The
-// 16-term chains run as packed fma.rn.f32x2 over head pairs: two independent IEEE FMAs each.
+// The query pairs of each lane stay in registers; the lane layout and the operation order of the exact
+// score are those of score.cuh.
 // ------------------------------------------------------------------------------------------------
 constexpr int kScoreWarps = 8;
 constexpr int kScoreThreads = kScoreWarps * 32;
@@ -50,8 +46,6 @@ struct ScoreArgs {
     const int32_t *pool_count;
     int pool_cap;
     int items_per_seq;
-    const uint2 *list;          // list mode: entries (b, block), count in *list_count
-    const int32_t *list_count;
     float *scores;
     int score_stride;
     void *ws;
@@ -74,72 +68,12 @@ struct ScoreSmem {
     int abort_flag;
 };
 
-__device__ __forceinline__ unsigned long long f2_pack(float lo, float hi)
-{
-    unsigned long long r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-
-__device__ __forceinline__ void f2_unpack(unsigned long long v, float &lo, float &hi)
-{
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-
-__device__ __forceinline__ unsigned long long ffma2(unsigned long long a, unsigned long long b, unsigned long long c)
-{
-    unsigned long long d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-
-// Score of the key whose dims 16j..16j+15 this lane holds in kr.  q2[s2][t] = (q[h(2 s2)][16j+t],
-// q[h(2 s2+1)][16j+t]) with h(s) = s ^ j.
-__device__ __forceinline__ float score_key(const unsigned long long (&q2)[4][16], const float (&w)[8], uint4 kr,
-                                           int lane)
-{
-    unsigned long long k2[16];
-    const uint32_t kw[4] = {kr.x, kr.y, kr.z, kr.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t lo = e4m3x2_to_f16x2((uint16_t)(kw[i] & 0xFFFF));
-        const uint32_t hi = e4m3x2_to_f16x2((uint16_t)(kw[i] >> 16));
-        const float k0 = h_lo(lo), k1 = h_hi(lo), k2v = h_lo(hi), k3 = h_hi(hi);
-        k2[4 * i + 0] = f2_pack(k0, k0);
-        k2[4 * i + 1] = f2_pack(k1, k1);
-        k2[4 * i + 2] = f2_pack(k2v, k2v);
-        k2[4 * i + 3] = f2_pack(k3, k3);
-    }
-    float p[8];
-#pragma unroll
-    for (int s2 = 0; s2 < 4; ++s2) {
-        unsigned long long acc = 0ull;   // (+0, +0)
-#pragma unroll
-        for (int t = 0; t < 16; ++t) acc = ffma2(q2[s2][t], k2[t], acc);
-        f2_unpack(acc, p[2 * s2], p[2 * s2 + 1]);
-    }
-    float a[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) a[i] = __fadd_rn(p[i], __shfl_xor_sync(0xffffffffu, p[4 + i], 4));
-    float c[2];
-#pragma unroll
-    for (int i = 0; i < 2; ++i) c[i] = __fadd_rn(a[i], __shfl_xor_sync(0xffffffffu, a[2 + i], 2));
-    const float d = __fadd_rn(c[0], __shfl_xor_sync(0xffffffffu, c[1], 1));
-    const float r = d > 0.f ? d : 0.f;
-    float score = 0.f;
-    const int base = lane & ~7;
-#pragma unroll
-    for (int h = 0; h < 8; ++h) score = __fmaf_rn(w[h], __shfl_sync(0xffffffffu, r, base | h), score);
-    return score;
-}
-
 __global__ void __launch_bounds__(kScoreThreads, 1) block_score_kernel(ScoreArgs a)
 {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     ScoreSmem &sm = *reinterpret_cast<ScoreSmem *>(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long total =
-        a.list ? ((long long)max(*a.list_count, 0) + kScoreWarps - 1) / kScoreWarps : (long long)a.B * a.items_per_seq;
+    const long long total = (long long)a.B * a.items_per_seq;
     // each CTA takes a contiguous range of items, so consecutive items mostly share a sequence (and
     // its query stays in registers)
     const long long per = (total + gridDim.x - 1) / gridDim.x;
@@ -159,33 +93,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) block_score_kernel(ScoreArgs
         const long long k = k0 + lane;
         const long long item = first + k;
         ItemMeta m{nullptr, 0, 0, kBlkEmpty, 0};
-        if (a.list) {
-            const long long e = item * kScoreWarps + warp;
-            if (item < last && e < *a.list_count) {
-                const uint2 ent = a.list[e];
-                const int b = (int)ent.x;
-                int blk = (int)ent.y;
-                const int L = (b >= 0 && b < a.B) ? a.seq_len[b] : 0;
-                const int nb = (L + kBlock - 1) / kBlock;
-                if (b < 0 || b >= a.B || blk < 0 || blk >= a.score_stride) {
-                    report(a.ws, CSA_ERR_DEVICE_DATA, e);
-                    sm.meta[warp][k % kMetaRing] = m;
-                    return;
-                }
-                m.b = b;
-                m.L = L;
-                m.v = blk;
-                const bool ok = L >= 1 && L <= a.max_seq_len && blk >= 0 && blk < nb;
-                const int page = ok ? a.block_table[(size_t)b * a.max_pages + blk / kBlocksPerPage] : -1;
-                if (page < 0 || page >= a.num_pages) {
-                    report(a.ws, CSA_ERR_DEVICE_DATA, e);
-                    blk = kBlkBad;
-                } else {
-                    m.src = a.keys + ((size_t)page * kPage + (size_t)(blk % kBlocksPerPage) * kBlock) * kIdxDim;
-                }
-                m.blk = blk;
-            }
-        } else if (item < last) {
+        if (item < last) {
             const int b = (int)(item / a.items_per_seq);
             const int grp = (int)(item % a.items_per_seq);
             const int L = a.seq_len[b];
@@ -286,8 +194,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1) block_score_kernel(ScoreArgs
             const uint8_t *sp = sm.stage[warp][st];
             const uint4 kr0 = *reinterpret_cast<const uint4 *>(sp + g * kIdxDim + 16 * j);
             const uint4 kr1 = *reinterpret_cast<const uint4 *>(sp + (4 + g) * kIdxDim + 16 * j);
-            const float s0 = score_key(q2, w, kr0, lane);
-            const float s1 = score_key(q2, w, kr1, lane);
+            const float s0 = score_key(QRegs{q2}, w, kr0, lane);
+            const float s1 = score_key(QRegs{q2}, w, kr1, lane);
             float best = -INFINITY;
             if (m.blk * kBlock + g < m.L) best = fmaxf(best, s0);   // a NaN score never wins
             if (m.blk * kBlock + 4 + g < m.L) best = fmaxf(best, s1);
@@ -470,45 +378,10 @@ cudaError_t launch_block_scores_full_or_pool(const uint8_t *keys, int num_pages,
     a.pool_cap = pool_cap;
     a.items_per_seq = pool ? (pool_cap + kScoreWarps - 1) / kScoreWarps
                            : (bt.max_seq_len + kPage - 1) / kPage;
-    a.list = nullptr;
-    a.list_count = nullptr;
     a.scores = scores;
     a.score_stride = score_stride;
     a.ws = ws;
     return launch_block_scores(a, st);
-}
-
-// Exact scores of the blocks named by a device-built work list: entry (b, blk) scores block blk of
-// sequence b into scores[b][blk].  The list and count come from this library's own kernels (seq_len,
-// block table and pages are still checked).
-cudaError_t launch_block_scores_list(const uint8_t *keys, int num_pages, const csa_batch &bt, const uint16_t *iq,
-                                     const float *iw, const uint2 *list, const int32_t *list_count, float *scores,
-                                     int score_stride, void *ws, cudaStream_t st)
-{
-    ScoreArgs a;
-    a.keys = keys;
-    a.num_pages = num_pages;
-    a.seq_len = bt.seq_len;
-    a.block_table = bt.block_table;
-    a.max_pages = bt.max_pages;
-    a.max_seq_len = bt.max_seq_len;
-    a.B = bt.B;
-    a.iq = iq;
-    a.iw = iw;
-    a.pool = nullptr;
-    a.pool_count = nullptr;
-    a.pool_cap = 0;
-    a.items_per_seq = 0;
-    a.list = list;
-    a.list_count = list_count;
-    a.scores = scores;
-    a.score_stride = score_stride;
-    a.ws = ws;
-    const size_t smem = sizeof(ScoreSmem);
-    cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void *>(block_score_kernel), smem);
-    if (e != cudaSuccess) return e;
-    block_score_kernel<<<num_sms(), kScoreThreads, smem, st>>>(a);
-    return cudaGetLastError();
 }
 
 cudaError_t launch_topk(const float *scores, int score_stride, const int32_t *seq_len, int max_seq_len,

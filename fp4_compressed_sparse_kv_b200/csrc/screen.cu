@@ -16,10 +16,9 @@
 //     head values d^_h = ((D_1 + D_2) + D_3) 2^-s, the approximate score t^ = the same weighted ReLU
 //     chain as the exact score, the bound eps_p, then per block the largest lower and upper bound,
 //     and a per-sequence histogram of the lower bounds.
-//  3. classify_a/b_kernel: thresholds T and U from the histograms and the widest interval, then each
-//     block is out, sure (certainly in the Top-K) or uncertain; uncertain blocks go to a work list.
-//  4. (indexer.cu) the exact scorer scores the uncertain blocks.
-//  5. finalize_kernel: the sure blocks plus the best uncertain ones, in ascending block order.
+//  3. (select.cu) from the bounds, the blocks sure to be in the Top-K, those that cannot be, and the
+//     uncertain rest, which are scored exactly; the sure blocks plus the best uncertain ones, in
+//     ascending block order.
 
 // The bound, with u = 2^-24, gamma_n = n u / (1 - n u), kmax_p the position's largest |key|:
 //  * exact chain: 16-term FMA chains then a 3-level tree; every product bf16 x E4M3 is exact in
@@ -45,7 +44,6 @@
 #include "common.cuh"
 #include "convert.cuh"
 #include "pipeline.cuh"
-#include "radix.cuh"
 #include "tcgen05.cuh"
 
 namespace csa {
@@ -89,18 +87,15 @@ static_assert(sizeof(QMeta) <= kQmBytes, "QMeta must fit its workspace slot");
 // ------------------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) qterm_kernel(const uint16_t *__restrict__ iq, const float *__restrict__ iw,
                                                     uint8_t *__restrict__ qt, QMeta *__restrict__ qm,
-                                                    int32_t *__restrict__ list_count, uint32_t *__restrict__ hist,
-                                                    uint32_t *__restrict__ hist2, uint32_t *__restrict__ seq_words)
+                                                    uint32_t *__restrict__ hist, uint32_t *__restrict__ hist2)
 {
     const int b = blockIdx.x, h = threadIdx.x >> 5, l = threadIdx.x & 31;
     grid_dep_launch();   // the screen may start streaming keys meanwhile
-    // the counters the later steps accumulate into start from zero on every call
-    if (b == 0 && threadIdx.x == 0 && list_count) *list_count = 0;
+    // the histograms the later steps accumulate into start from zero on every call
     for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) {
         hist[(size_t)b * kHistBins + i] = 0u;
         if (hist2) hist2[(size_t)b * kHistBins + i] = 0u;
     }
-    if (seq_words && threadIdx.x < kTopkWords) seq_words[(size_t)b * kTopkWords + threadIdx.x] = 0u;
     const uint2 raw = reinterpret_cast<const uint2 *>(iq + ((size_t)b * kIdxHeads + h) * kIdxDim)[l];
     const float q[4] = {bf16_lo(raw.x), bf16_hi(raw.x), bf16_lo(raw.y), bf16_hi(raw.y)};
     float amax = 0.f;
@@ -503,356 +498,6 @@ __global__ void __launch_bounds__(kScrThreads, 1) screen_kernel(const __grid_con
 }
 
 // ------------------------------------------------------------------------------------------------
-// Step 3: classification, over a grid of (chunk, sequence) CTAs.  With T <= the k-th largest lower
-// bound and U >= the (k+1)-th largest upper bound, a block is
-//   out        if upper < T: k blocks have lower >= T, so k scores are >= T, above this one's;
-//   sure       if lower > U: only blocks with upper > U, at most k of them and this block among
-//              them, can reach its score, so it is in the Top-K whatever the ties;
-//   uncertain  otherwise: scored exactly afterwards.
-// The k-th largest lower-bound key X is located to 24 bits: its top 12 bits from the screen's
-// per-sequence histogram, the next 12 from a second histogram of the keys in that bin (pass A).
-// T = X with the last 8 bits clear; U = (X with them set) + the widest interval of the sequence,
-// rounded up (pass A takes that maximum too): a block with upper > U has lower > X, and fewer than k
-// blocks do.  If some bound of the sequence is not finite, U is the largest key: no block is sure.
-// Pass B writes every block's class and appends the uncertain blocks to the sequence's slice and to
-// the global re-scoring work list.
-// ------------------------------------------------------------------------------------------------
-constexpr int kClsThreads = 256;
-constexpr uint8_t kOut = 0, kSure = 1, kUncertain = 2, kChosen = 3, kTie = 4;
-
-// Per-sequence words: sure blocks, uncertain blocks, order key of the widest interval, and the
-// first-level histogram bin of the k-th largest lower bound with that element's rank inside it.
-struct SeqWords {
-    uint32_t n_sure, n_uncertain, wmax_key, bin1, r1, pad[3];
-};
-static_assert(sizeof(SeqWords) == kTopkWords * 4, "SeqWords fills one sequence's select words");
-
-// Over a kHistBins-bin histogram h: the bin holding the rank-th largest element (1-based) and that
-// element's rank inside the bin; every thread gets both.  If the counts fall short of rank: bin 0
-// (a threshold that keeps everything).
-template <int kThreads>
-__device__ __forceinline__ void rank_bin(const uint32_t *h, uint32_t rank, uint32_t *scratch, int *bin_out,
-                                         uint32_t *rank_out)
-{
-    constexpr int kPer = kHistBins / kThreads;
-    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    if (t == 0) {
-        scratch[33] = 0u;
-        scratch[34] = 1u;
-    }
-    // thread t owns the kPer bins below kHistBins - kPer t, largest first
-    uint32_t c[kPer], s = 0;
-#pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-        c[i] = h[kHistBins - 1 - kPer * t - i];
-        s += c[i];
-    }
-    uint32_t x = s;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) scratch[warp] = x;
-    __syncthreads();
-    uint32_t before = 0;
-    for (int wi = 0; wi < warp; ++wi) before += scratch[wi];
-    uint32_t run = before + x - s;   // elements in larger bins than this thread's
-    if (run < rank && rank <= run + s) {
-#pragma unroll
-        for (int i = 0; i < kPer; ++i) {
-            if (run < rank && rank <= run + c[i]) {
-                scratch[33] = (uint32_t)(kHistBins - 1 - kPer * t - i);
-                scratch[34] = rank - run;
-            }
-            run += c[i];
-        }
-    }
-    __syncthreads();
-    *bin_out = (int)scratch[33];
-    *rank_out = scratch[34];
-    __syncthreads();
-}
-
-struct ClsArgs {
-    const float *lo;
-    const float *hi;
-    int stride;          // row stride of lo, hi and uslice (blocks)
-    int sstride;         // row stride of status (bytes, a multiple of 16)
-    const int32_t *seq_len;
-    int max_seq_len;
-    int k;
-    const uint32_t *hist;
-    uint32_t *hist2;
-    SeqWords *words;
-    uint8_t *status;
-    int32_t *uslice;
-    uint2 *list;
-    int32_t *list_count;
-    void *ws;
-};
-
-__device__ __forceinline__ bool cls_chunk(const ClsArgs &a, int b, int &n, int &i0, int &i1)
-{
-    const int L = a.seq_len[b];
-    if (L < 1 || L > a.max_seq_len) return false;
-    n = (L + kBlock - 1) / kBlock;
-    if (n <= a.k) return false;   // every block is selected
-    const int per = (n + gridDim.x - 1) / gridDim.x;
-    i0 = blockIdx.x * per;
-    i1 = min(n, i0 + per);
-    return i0 < i1;
-}
-
-__global__ void __launch_bounds__(kClsThreads) classify_a_kernel(const ClsArgs a)
-{
-    __shared__ uint32_t scratch[40];
-    const int b = blockIdx.y;
-    if (blockIdx.x == 0 && threadIdx.x == 0) {
-        const int L = a.seq_len[b];
-        if (L < 1 || L > a.max_seq_len) report(a.ws, CSA_ERR_DEVICE_DATA, b);
-    }
-    int n, i0, i1;
-    if (!cls_chunk(a, b, n, i0, i1)) return;
-    int bin1;
-    uint32_t r1;
-    rank_bin<kClsThreads>(a.hist + (size_t)b * kHistBins, (uint32_t)a.k, scratch, &bin1, &r1);
-    if (blockIdx.x == 0 && threadIdx.x == 0) {
-        a.words[b].bin1 = (uint32_t)bin1;
-        a.words[b].r1 = r1;
-    }
-    const float *lp = a.lo + (size_t)b * a.stride;
-    const float *hp = a.hi + (size_t)b * a.stride;
-    uint32_t *h2 = a.hist2 + (size_t)b * kHistBins;
-    uint32_t wkey = 0u;   // order key of the widest interval (+inf when a bound is not finite)
-    for (int i = i0 + threadIdx.x; i < i1; i += kClsThreads) {
-        const float l = lp[i], h = hp[i];
-        const float w = __fsub_ru(h, l);
-        wkey = max(wkey, w == w ? order_key(w) : 0xFF800000u);
-        const uint32_t kl = order_key(l);
-        if ((int)(kl >> 20) == bin1) atomicAdd(&h2[(kl >> 8) & (kHistBins - 1)], 1u);
-    }
-    wkey = block_reduce_minmax(wkey, true, scratch);
-    if (threadIdx.x == 0) atomicMax(&a.words[b].wmax_key, wkey);
-}
-
-__global__ void __launch_bounds__(kClsThreads) classify_b_kernel(const ClsArgs a)
-{
-    __shared__ uint32_t scratch[40];
-    const int b = blockIdx.y, lane = threadIdx.x & 31;
-    int n, i0, i1;
-    if (!cls_chunk(a, b, n, i0, i1)) return;
-    const int bin1 = (int)a.words[b].bin1;
-    int bin2;
-    uint32_t r2;
-    rank_bin<kClsThreads>(a.hist2 + (size_t)b * kHistBins, a.words[b].r1, scratch, &bin2, &r2);
-    const uint32_t T = ((uint32_t)bin1 << 20) | ((uint32_t)bin2 << 8);
-    const uint32_t wkey = a.words[b].wmax_key;
-    const float wmax = key_to_float(wkey);
-    const uint32_t U = wkey >= 0xFF800000u ? 0xFFFFFFFFu : order_key(__fadd_ru(key_to_float(T | 0xFFu), wmax));
-    const float *lp = a.lo + (size_t)b * a.stride;
-    const float *hp = a.hi + (size_t)b * a.stride;
-    uint8_t *stat = a.status + (size_t)b * a.sstride;
-    int32_t *us = a.uslice + (size_t)b * a.stride;
-    const uint32_t lt = (1u << lane) - 1u;
-    uint32_t n_sure = 0;
-    for (int base = i0 + (threadIdx.x & ~31); base < i1; base += kClsThreads) {
-        const int i = base + lane;
-        uint8_t c = kOut;
-        if (i < i1) {
-            const uint32_t hk = order_key(hp[i]), lk = order_key(lp[i]);
-            c = hk < T ? kOut : (lk > U ? kSure : kUncertain);
-            stat[i] = c;
-        }
-        n_sure += c == kSure;
-        // uncertain blocks: one atomic per warp for the slice and one for the work list
-        const uint32_t bu = __ballot_sync(0xffffffffu, c == kUncertain);
-        if (bu) {
-            uint32_t sbase = 0, lbase = 0;
-            if (lane == 0) {
-                sbase = atomicAdd(&a.words[b].n_uncertain, (uint32_t)__popc(bu));
-                lbase = (uint32_t)atomicAdd(a.list_count, __popc(bu));
-            }
-            sbase = __shfl_sync(0xffffffffu, sbase, 0);
-            lbase = __shfl_sync(0xffffffffu, lbase, 0);
-            if (c == kUncertain) {
-                const uint32_t r = __popc(bu & lt);
-                us[sbase + r] = i;
-                a.list[lbase + r] = make_uint2((uint32_t)b, (uint32_t)i);
-            }
-        }
-    }
-    n_sure = block_reduce_sum(n_sure, scratch);
-    if (threadIdx.x == 0 && n_sure) atomicAdd(&a.words[b].n_sure, n_sure);
-}
-
-// ------------------------------------------------------------------------------------------------
-// Step 5 (after the exact re-scoring of the uncertain blocks): the sure blocks plus the
-// k - n_sure best uncertain ones by exact score (larger first, then lower block id), written in
-// ascending block order.  One CTA per sequence.  The chosen uncertain blocks are found on the
-// sequence's slice -- by counting each one's rank when there are few, else by radix selection, whose
-// blocks tied at the threshold are marked and the lowest-numbered need_eq of them taken -- and marked
-// in the status bytes; one ordered pass over the status bytes writes the result.
-// ------------------------------------------------------------------------------------------------
-constexpr int kFinThreads = 1024;
-constexpr int kFinWarps = kFinThreads / 32;
-constexpr int kFinCache = 16384;         // uncertain keys cached up to this many
-constexpr int kFinRankMax = 512;         // up to this many uncertain blocks: rank by counting
-constexpr int kFinStatusCache = 65536;   // status bytes staged in shared memory up to this many blocks
-
-__global__ void __launch_bounds__(kFinThreads, 1) finalize_kernel(
-    const float *__restrict__ scores, int score_stride, const int32_t *__restrict__ seq_len, int max_seq_len,
-    uint8_t *__restrict__ status, int sstride, const int32_t *__restrict__ uslice, const SeqWords *__restrict__ words,
-    int stride, int k, int32_t *__restrict__ out_blocks, int32_t *__restrict__ out_count, void *ws)
-{
-    extern __shared__ uint32_t fz_smem[];
-    uint32_t *whist = fz_smem;                    // [32 warps][256]
-    uint32_t *skeys = whist + kFinWarps * 256;    // keys of the uncertain blocks
-    int32_t *sblk = reinterpret_cast<int32_t *>(skeys + kFinRankMax);   // their ids (rank path)
-    uint8_t *sstat = reinterpret_cast<uint8_t *>(skeys + kFinCache);    // staged status bytes
-    __shared__ uint32_t scratch[72];
-    __shared__ uint32_t sel[2];
-    const int b = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    grid_dep_launch();   // the attention may be scheduled meanwhile
-    const int L = seq_len[b];
-    int32_t *out = out_blocks + (size_t)b * k;
-    if (L < 1 || L > max_seq_len) {   // reported by the classification
-        if (t == 0) out_count[b] = 0;
-        return;
-    }
-    const int n = (L + kBlock - 1) / kBlock;
-    if (n <= k) {   // every block is selected
-        for (int i = t; i < n; i += kFinThreads) out[i] = i;
-        if (t == 0) out_count[b] = n;
-        return;
-    }
-    const SeqWords sw = words[b];
-    const int n_sure = (int)sw.n_sure, nu = (int)sw.n_uncertain;
-    const int kk = k - n_sure;   // how many uncertain blocks to take
-    if (n_sure > k || kk > nu) {
-        if (t == 0) {
-            out_count[b] = 0;
-            report(ws, CSA_ERR_DEVICE_DATA, (long long)b);
-        }
-        return;
-    }
-    const float *sc = scores + (size_t)b * score_stride;
-    const int32_t *us = uslice + (size_t)b * stride;
-    uint8_t *stat = status + (size_t)b * sstride;
-    const bool staged = n <= kFinStatusCache;
-    if (staged) {   // status row into shared memory, 16 bytes per load
-        const int nv = (n + 15) >> 4;
-        for (int i = t; i < nv; i += kFinThreads)
-            reinterpret_cast<uint4 *>(sstat)[i] = reinterpret_cast<const uint4 *>(stat)[i];
-    }
-    uint8_t *st8 = staged ? sstat : stat;
-    uint32_t need_eq = 0;
-    if (kk > 0 && kk == nu) {
-        __syncthreads();
-        for (int j = t; j < nu; j += kFinThreads) st8[us[j]] = kChosen;
-    } else if (kk > 0 && nu <= kFinRankMax) {
-        for (int j = t; j < nu; j += kFinThreads) {
-            const int blk = us[j];
-            sblk[j] = blk;
-            skeys[j] = order_key(sc[blk]);
-        }
-        __syncthreads();
-        // warp per uncertain block, its lanes splitting the comparisons
-        for (int j = warp; j < nu; j += kFinWarps) {
-            const uint32_t u = skeys[j];
-            const int bj = sblk[j];
-            int rank = 0;
-            for (int i = lane; i < nu; i += 32) {
-                const uint32_t x = skeys[i];
-                rank += (x > u) || (x == u && sblk[i] < bj);
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) rank += __shfl_xor_sync(0xffffffffu, rank, o);
-            if (lane == 0 && rank < kk) st8[bj] = kChosen;
-        }
-    } else if (kk > 0) {
-        const bool cached = nu <= kFinCache;
-        if (cached)
-            for (int j = t; j < nu; j += kFinThreads) skeys[j] = order_key(sc[us[j]]);
-        __syncthreads();
-        auto key = [&](int j) { return cached ? skeys[j] : order_key(sc[us[j]]); };
-        uint32_t T;
-        radix_select<kFinThreads>(nu, (uint32_t)kk, key, 0, whist, scratch, sel, T, need_eq);
-        for (int j = t; j < nu; j += kFinThreads) {
-            const uint32_t u = key(j);
-            if (u > T) st8[us[j]] = kChosen;
-            else if (u == T) st8[us[j]] = kTie;
-        }
-    } else {
-        __syncthreads();
-    }
-    __syncthreads();
-    // ordered output: sure and chosen blocks, and the first need_eq tied ones.  Thread t owns the
-    // bytes [t c, t c + c), c a multiple of 16, read 16 at a time.
-    const int c = ((n + kFinThreads - 1) / kFinThreads + 15) & ~15;
-    const int i0 = min(n, t * c), i1 = min(n, i0 + c);
-    auto cls = [](uint32_t v, int j) { return (v >> (8 * j)) & 0xFFu; };
-    uint32_t n_take = 0, n_tie = 0;
-    for (int i = i0; i < i1; i += 16) {
-        const uint4 v = *reinterpret_cast<const uint4 *>(st8 + i);
-        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {
-            const uint32_t x = cls(w4[q >> 2], q & 3);
-            const bool in = i + q < i1;
-            n_take += in && (x == kSure || x == kChosen);
-            n_tie += in && x == kTie;
-        }
-    }
-    // exclusive scan of (n_take, n_tie) over the CTA
-    uint32_t x = n_take, y = n_tie;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t xa = __shfl_up_sync(0xffffffffu, x, o), ya = __shfl_up_sync(0xffffffffu, y, o);
-        if (lane >= o) {
-            x += xa;
-            y += ya;
-        }
-    }
-    if (lane == 31) {
-        scratch[warp] = x;
-        scratch[32 + warp] = y;
-    }
-    __syncthreads();
-    uint32_t r_take = x - n_take, r_tie = y - n_tie, total = 0, total_tie = 0;
-    for (int wi = 0; wi < kFinWarps; ++wi) {
-        const uint32_t a0 = scratch[wi], a1 = scratch[32 + wi];
-        if (wi < warp) {
-            r_take += a0;
-            r_tie += a1;
-        }
-        total += a0;
-        total_tie += a1;
-    }
-    for (int i = i0; i < i1; i += 16) {
-        const uint4 v = *reinterpret_cast<const uint4 *>(st8 + i);
-        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {
-            if (i + q >= i1) break;
-            const uint32_t xq = cls(w4[q >> 2], q & 3);
-            if (xq == kSure || xq == kChosen) {
-                const uint32_t pos = r_take + min(r_tie, need_eq);
-                if (pos < (uint32_t)k) out[pos] = i + q;
-                ++r_take;
-            } else if (xq == kTie) {
-                if (r_tie < need_eq && r_take + r_tie < (uint32_t)k) out[r_take + r_tie] = i + q;
-                ++r_tie;
-            }
-        }
-    }
-    if (t == 0) {
-        out_count[b] = k;
-        if (total + min(total_tie, need_eq) != (uint32_t)k) report(ws, CSA_ERR_DEVICE_DATA, (long long)b);
-    }
-}
-
-// ------------------------------------------------------------------------------------------------
 // Host side
 // ------------------------------------------------------------------------------------------------
 namespace {
@@ -935,16 +580,14 @@ int sm_count()
 bool screen_supported(int num_pages) { return (long long)num_pages * kPage <= 0xFFFFFFFFll; }
 
 cudaError_t launch_screen_bounds(const uint8_t *keys, int num_pages, const csa_batch &bt, const uint16_t *iq,
-                                 const float *iw, uint8_t *qt, void *qm, int32_t *list_count, uint32_t *hist,
-                                 uint32_t *hist2, void *words, float *lo, float *hi, int stride, void *ws,
-                                 cudaStream_t st)
+                                 const float *iw, uint8_t *qt, void *qm, uint32_t *hist, uint32_t *hist2, float *lo,
+                                 float *hi, int stride, void *ws, cudaStream_t st)
 {
     cudaError_t e;
     CUtensorMap map;
     if ((e = keys_tensor_map(keys, num_pages, &map)) != cudaSuccess) return e;
 
-    qterm_kernel<<<bt.B, 256, 0, st>>>(iq, iw, qt, reinterpret_cast<QMeta *>(qm), list_count, hist, hist2,
-                                       reinterpret_cast<uint32_t *>(words));
+    qterm_kernel<<<bt.B, 256, 0, st>>>(iq, iw, qt, reinterpret_cast<QMeta *>(qm), hist, hist2);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     ScreenArgs sa;
@@ -970,54 +613,6 @@ cudaError_t launch_screen_bounds(const uint8_t *keys, int num_pages, const csa_b
     if ((e = allow_dynamic_smem(reinterpret_cast<const void *>(screen_kernel), smem)) != cudaSuccess)
         return e;
     return launch_overlapped(screen_kernel, dim3(grid), dim3(kScrThreads), smem, st, map, sa);
-}
-
-cudaError_t launch_classify(const float *lo, const float *hi, int stride, const csa_batch &bt, int k,
-                            const uint32_t *hist, uint32_t *hist2, void *words, uint8_t *status, int sstride,
-                            int32_t *uslice, uint2 *list, int32_t *list_count, void *ws, cudaStream_t st)
-{
-    ClsArgs a;
-    a.lo = lo;
-    a.hi = hi;
-    a.stride = stride;
-    a.sstride = sstride;
-    a.seq_len = bt.seq_len;
-    a.max_seq_len = bt.max_seq_len;
-    a.k = k;
-    a.hist = hist;
-    a.hist2 = hist2;
-    a.words = reinterpret_cast<SeqWords *>(words);
-    a.status = status;
-    a.uslice = uslice;
-    a.list = list;
-    a.list_count = list_count;
-    a.ws = ws;
-    // about two CTAs per SM over the batch, at least 512 blocks per chunk
-    const int nb = (bt.max_seq_len + kBlock - 1) / kBlock;
-    int chunks = (2 * sm_count() + bt.B - 1) / bt.B;
-    const int max_chunks = (nb + 511) / 512;
-    if (chunks > max_chunks) chunks = max_chunks;
-    if (chunks < 1) chunks = 1;
-    const dim3 grid(chunks, bt.B);
-    classify_a_kernel<<<grid, kClsThreads, 0, st>>>(a);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    classify_b_kernel<<<grid, kClsThreads, 0, st>>>(a);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_finalize(const float *scores, int score_stride, const csa_batch &bt, uint8_t *status,
-                            int sstride, const int32_t *uslice, const void *words, int stride, int k,
-                            int32_t *out_blocks, int32_t *out_count, void *ws, cudaStream_t st)
-{
-    const size_t smem = ((size_t)kFinWarps * 256 + kFinCache) * 4 + kFinStatusCache;
-    static_assert(2 * kFinRankMax <= kFinCache, "rank-path keys and ids share the key cache");
-    cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void *>(finalize_kernel), smem);
-    if (e != cudaSuccess) return e;
-    finalize_kernel<<<bt.B, kFinThreads, smem, st>>>(scores, score_stride, bt.seq_len, bt.max_seq_len, status, sstride,
-                                                      uslice, reinterpret_cast<const SeqWords *>(words), stride, k,
-                                                      out_blocks, out_count, ws);
-    return cudaGetLastError();
 }
 
 }  // namespace csa

@@ -265,3 +265,21 @@ def test_bounds_bracket_exact_scores_under_slice_cancellation():
     for b, L in enumerate(lens):
         exact = oracle.block_scores(iq[b], iw[b], keys[b])
         assert got[b].tolist() == oracle.topk(np.arange(len(exact), dtype=np.int32), exact, k).tolist()
+
+
+@pytest.mark.parametrize("rows", [1, 3])
+def test_long_sequence_of_few_distinct_keys(rows):
+    """200,003 positions (25,001 blocks) whose keys take only `rows` distinct values: every block is
+    uncertain or tied, each CTA of the selection holds more uncertain blocks than its shared-memory
+    list, and the k-th score is shared by thousands of blocks, of which the lowest-numbered must be
+    taken.  The selection must equal the oracle's Top-K."""
+    rng = np.random.default_rng([15, rows])
+    L, k = 200003, 3000
+    base = keys_for(rng, "gauss", rows)
+    keys = [base[rng.integers(0, rows, L)] if rows > 1 else np.tile(base, (L, 1)), keys_for(rng, "gauss", 999)]
+    iq, iw = synth.index_query(rng, 2)
+    layer, batch = gpu_layer(keys, 10)
+    got = full_select(layer, batch, iq, iw, k)
+    for b in range(2):
+        exact = oracle.block_scores(iq[b], iw[b], keys[b])
+        assert got[b].tolist() == oracle.topk(np.arange(len(exact), dtype=np.int32), exact, k).tolist(), b
