@@ -28,7 +28,7 @@ cudaError_t launch_screen_bounds(const uint8_t *keys, int num_pages, const csa_b
                                  float *hi, int stride, void *ws, cudaStream_t st);
 cudaError_t launch_select(const float *lo, const float *hi, int lstride, const csa_batch &bt, int k,
                           const uint32_t *hist, uint32_t *hist2, uint8_t *status, int sstride, int32_t *uslice,
-                          uint32_t *okeys, int ustride, uint32_t *takes, const uint8_t *keys, int num_pages,
+                          uint32_t *okeys, int ustride, const uint8_t *keys, int num_pages,
                           const uint16_t *iq, const float *iw, int32_t *out_blocks, int32_t *out_count, void *ws,
                           cudaStream_t st);
 cudaError_t launch_attn_tc(const AttnArgs &a, cudaStream_t st);
@@ -217,8 +217,8 @@ csa_status csa_indexer_full(const csa_kv_layer *layer, const csa_batch *batch, c
                                          lstride, ws, st);
     if (e == cudaSuccess)   // the score region (B x score_cap >= B x nb words) keeps the overflow keys
         e = launch_select(lo, hi, lstride, *batch, k, hist, hist2, status, (int)w.status_stride, uslice,
-                          reinterpret_cast<uint32_t *>(scores), nb, reinterpret_cast<uint32_t *>(base + w.topk),
-                          layer->keys, layer->num_pages, iq, iw, out_blocks, out_count, ws, st);
+                          reinterpret_cast<uint32_t *>(scores), nb, layer->keys, layer->num_pages, iq, iw,
+                          out_blocks, out_count, ws, st);
     return cuda_status(e);
 }
 

@@ -208,6 +208,15 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const float *__restri
     __shared__ float red[8];
     const int h = blockIdx.x, b = blockIdx.y, t = threadIdx.x, lane = t & 31, warp = t >> 5;
     grid_dep_wait();   // every split's partial
+    // the partials of the first kPre splits are loaded at once, before (and independently of) the
+    // split weights, so that the whole read is one round trip
+    constexpr int kPre = 24;
+    const float4 *po = reinterpret_cast<const float4 *>(part_o + ((size_t)b * splits * H + h) * kLatent) + t;
+    const size_t stride = (size_t)H * kLatent / 4;
+    float4 pre[kPre];
+#pragma unroll
+    for (int q = 0; q < kPre; ++q)
+        if (q < splits) pre[q] = po[(size_t)q * stride];
     const float2 *ml = part_ml + (size_t)b * splits * H + h;
     float M = -INFINITY;
     for (int s = t; s < splits; s += 128) M = fmaxf(M, ml[(size_t)s * H].x);
@@ -229,24 +238,18 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const float *__restri
     if (lane == 0) red[4 + warp] = den;
     __syncthreads();
     den = red[4] + red[5] + red[6] + red[7];
-    const float4 *po = reinterpret_cast<const float4 *>(part_o + ((size_t)b * splits * H + h) * kLatent) + t;
-    const size_t stride = (size_t)H * kLatent / 4;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    int s = 0;
-    for (; s + 4 <= splits; s += 4) {
-        float4 o[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) o[q] = po[(size_t)(s + q) * stride];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const float wv = wgt[s + q];
-            acc.x = fmaf(wv, o[q].x, acc.x);
-            acc.y = fmaf(wv, o[q].y, acc.y);
-            acc.z = fmaf(wv, o[q].z, acc.z);
-            acc.w = fmaf(wv, o[q].w, acc.w);
+    for (int q = 0; q < kPre; ++q) {
+        if (q < splits) {
+            const float wv = wgt[q];
+            acc.x = fmaf(wv, pre[q].x, acc.x);
+            acc.y = fmaf(wv, pre[q].y, acc.y);
+            acc.z = fmaf(wv, pre[q].z, acc.z);
+            acc.w = fmaf(wv, pre[q].w, acc.w);
         }
     }
-    for (; s < splits; ++s) {
+    for (int s = kPre; s < splits; ++s) {
         const float4 o = po[(size_t)s * stride];
         const float wv = wgt[s];
         acc.x = fmaf(wv, o.x, acc.x);

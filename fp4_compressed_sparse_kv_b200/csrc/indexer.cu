@@ -89,8 +89,9 @@ __global__ void __launch_bounds__(kScoreThreads, 1) block_score_kernel(ScoreArgs
     __syncthreads();
 
     // ---- metadata of this warp's block of items k0 .. k0+31, one item per lane, loads in parallel
-    auto resolve32 = [&](long long k0) {
-        const long long k = k0 + lane;
+    // local item counters are 32-bit (stage and ring arithmetic by constants stays cheap)
+    auto resolve32 = [&](uint32_t k0) {
+        const uint32_t k = k0 + lane;
         const long long item = first + k;
         ItemMeta m{nullptr, 0, 0, kBlkEmpty, 0};
         if (item < last) {
@@ -134,7 +135,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) block_score_kernel(ScoreArgs
         sm.meta[warp][k % kMetaRing] = m;
     };
     // lane 0: start the copy of item k's block into stage k % kScoreStages
-    auto issue = [&](long long k) {
+    auto issue = [&](uint32_t k) {
         const long long item = first + k;
         if (item >= last) return;
         const int st = (int)(k % kScoreStages);
@@ -151,16 +152,16 @@ __global__ void __launch_bounds__(kScoreThreads, 1) block_score_kernel(ScoreArgs
     resolve32(0);
     __syncwarp();
     if (lane == 0)
-        for (long long k = 0; k < kScoreStages - 1; ++k) issue(k);
+        for (uint32_t k = 0; k < kScoreStages - 1; ++k) issue(k);
     __syncwarp();
 
     unsigned long long q2[4][16];
     float w[8];
     int cur_b = -1;
     const int g = lane >> 3, j = lane & 7;
-    long long k = 0;
+    uint32_t k = 0;
     for (long long item = first; item < last; ++item, ++k) {
-        const long long kn = k + kScoreStages - 1;   // the item whose copy starts now
+        const uint32_t kn = k + kScoreStages - 1;   // the item whose copy starts now
         if ((kn & 31) == 0) {
             resolve32(kn);
             __syncwarp();
@@ -210,7 +211,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1) block_score_kernel(ScoreArgs
     // no copy may still be landing in shared memory when the CTA exits: wait for every stage this
     // warp started (k counts the items consumed; issue() ran up to k + kScoreStages - 2)
     if (lane == 0) {
-        for (long long kk = k; kk < k + kScoreStages - 1; ++kk) {
+        for (uint32_t kk = k; kk < k + kScoreStages - 1; ++kk) {
             const long long item = first + kk;
             if (item >= last) break;
             volatile int no_abort = 0;

@@ -278,7 +278,9 @@ __global__ void __launch_bounds__(kScrThreads, 1) screen_kernel(const __grid_con
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long first = (long long)blockIdx.x * a.per_cta;
     const long long last = first + a.per_cta < a.total ? first + a.per_cta : a.total;
-    const long long n_items = last > first ? last - first : 0;
+    // local tile counters are 32-bit (at most 2^31 tiles per CTA): stage and phase arithmetic by
+    // constants then stays a few instructions
+    const uint32_t n_items = last > first ? (uint32_t)(last - first) : 0u;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kScrStages; ++s) {
@@ -305,8 +307,8 @@ __global__ void __launch_bounds__(kScrThreads, 1) screen_kernel(const __grid_con
 
     if (warp == 0) {
         // ---------------- loader ----------------
-        auto resolve32 = [&](long long k0) {
-            const long long k = k0 + lane;
+        auto resolve32 = [&](uint32_t k0) {
+            const uint32_t k = k0 + lane;
             ScrItem it{-1, 0, 0, -1, -1};
             if (k < n_items) {
                 const long long item = first + k;
@@ -338,9 +340,9 @@ __global__ void __launch_bounds__(kScrThreads, 1) screen_kernel(const __grid_con
             }
             sm.ring[k % kScrRing] = it;
         };
-        long long issued = 0;
+        uint32_t issued = 0;
         bool q_visible = false;   // the query terms of the previous grid have been waited for
-        for (long long k = 0; k < n_items; ++k) {
+        for (uint32_t k = 0; k < n_items; ++k) {
             if ((k & 31) == 0) {
                 resolve32(k);
                 __syncwarp();
@@ -375,7 +377,7 @@ __global__ void __launch_bounds__(kScrThreads, 1) screen_kernel(const __grid_con
         }
         // no copy may still be landing in shared memory when the CTA exits
         if (lane == 0) {
-            for (long long kk = issued > kScrStages ? issued - kScrStages : 0; kk < issued; ++kk) {
+            for (uint32_t kk = issued > kScrStages ? issued - kScrStages : 0u; kk < issued; ++kk) {
                 volatile int no_abort = 0;
                 mbar_wait(&sm.full[kk % kScrStages], (uint32_t)((kk / kScrStages) & 1), &no_abort, a.ws, 25);
             }
@@ -385,7 +387,7 @@ __global__ void __launch_bounds__(kScrThreads, 1) screen_kernel(const __grid_con
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
             bool any_mma = false;
-            for (long long k = 0; k < n_items; ++k) {
+            for (uint32_t k = 0; k < n_items; ++k) {
                 const int st = (int)(k % kScrStages), d = (int)(k % kScrAcc);
                 if (!mbar_wait(&sm.full[st], (uint32_t)((k / kScrStages) & 1), &sm.abort_flag, a.ws, 21)) break;
                 if (!mbar_wait(&sm.dfree[d], (uint32_t)(((k / kScrAcc) & 1) ^ 1), &sm.abort_flag, a.ws, 22)) break;
@@ -415,7 +417,7 @@ __global__ void __launch_bounds__(kScrThreads, 1) screen_kernel(const __grid_con
         // ---------------- row maxima, group mg: tiles k = mg, mg + 2, ...; thread = tile row ----------
         const int mg = (warp - 2) >> 2;
         const int r = threadIdx.x - 64 - 128 * mg;
-        for (long long k = mg; k < n_items; k += kScrMaxGroups) {
+        for (uint32_t k = mg; k < n_items; k += kScrMaxGroups) {
             const int st = (int)(k % kScrStages), d = (int)(k % kScrAcc);
             if (!warp_wait(&sm.full[st], (uint32_t)((k / kScrStages) & 1), &sm.abort_flag, a.ws, 27)) break;
             if (!warp_wait(&sm.dfree[d], (uint32_t)(((k / kScrAcc) & 1) ^ 1), &sm.abort_flag, a.ws, 28)) break;
@@ -434,7 +436,7 @@ __global__ void __launch_bounds__(kScrThreads, 1) screen_kernel(const __grid_con
         int cur_b = -1;
         QMeta qm{};
         float w[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (long long k = g; k < n_items; k += kScrEpiGroups) {
+        for (uint32_t k = g; k < n_items; k += kScrEpiGroups) {
             const int d = (int)(k % kScrAcc);
             if (!warp_wait(&sm.dfull[d], (uint32_t)((k / kScrAcc) & 1), &sm.abort_flag, a.ws, 24)) break;
             tc_fence_after();

@@ -61,7 +61,6 @@ struct SelArgs {
     int32_t *uslice;            // [B][ustride]: uncertain blocks beyond a CTA's shared-memory list
     uint32_t *okeys;            //   and their exact-score order keys
     int ustride;
-    uint32_t *takes;            // [B][kSelCtas]: blocks each CTA contributes to the result
     const int32_t *seq_len;
     int max_seq_len;
     const int32_t *block_table;
@@ -84,10 +83,11 @@ struct SelSmem {
     uint32_t gkey[kSelRankCap];              // the sequence's uncertain blocks (rank path)
     int32_t gid[kSelRankCap];
     alignas(16) uint8_t sstat[kSelStatCap];  // class bytes of the chunk
+    int32_t cpage[kSelRound / kBlocksPerPage];   // pages of the chunk's first round
     uint32_t rhist[2][256];                  // radix digits of this CTA's keys (read by the cluster)
     uint32_t scratch[40];
     uint32_t wkey;                           // this CTA's widest interval (read by the cluster)
-    uint32_t n_sure, n_unc, n_tie;           // this CTA's counts (read by the cluster)
+    uint32_t n_sure, n_unc, n_tie, n_take;   // this CTA's counts (read by the cluster)
     uint32_t n_chosen;
     uint32_t sel[2];
 };
@@ -161,6 +161,13 @@ __device__ __forceinline__ void rank_bin(const uint32_t *h, uint32_t rank, uint3
     __syncthreads();
 }
 
+// Split cluster barrier: arrive (no memory ordering) ... wait.
+__device__ __forceinline__ void cluster_arrive_relaxed()
+{
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
+
 // The 8 values p[i .. i+8) (i a multiple of 8 from a 16-byte aligned row), -inf past `end`.
 __device__ __forceinline__ void load8(const float *p, int i, int end, float (&v)[8])
 {
@@ -222,6 +229,8 @@ __global__ void __cluster_dims__(kSelCtas, 1, 1) __launch_bounds__(kSelThreads, 
     float l8[8], h8[8];
     load8(lp, i0 + kSelPer * t, i1, l8);   // round 0, in flight during the first rank_bin
     load8(hp, i0 + kSelPer * t, i1, h8);
+    static_assert(kSelRound / kBlocksPerPage == kSelThreads, "one page of round 0 per thread");
+    if (i0 + kBlocksPerPage * t < i1) sm.cpage[t] = btab[i0 / kBlocksPerPage + t];   // (i0: whole pages)
     int bin1;
     uint32_t r1;
     rank_bin(a.hist + (size_t)b * kHistBins, (uint32_t)a.k, sm.scratch, &bin1, &r1);
@@ -285,7 +294,7 @@ __global__ void __cluster_dims__(kSelCtas, 1, 1) __launch_bounds__(kSelThreads, 
                 const int blk = i + q;
                 if (pos < (uint32_t)kSelListCap) {
                     sm.uid[pos] = blk;
-                    sm.upage[pos] = btab[blk / kBlocksPerPage];
+                    sm.upage[pos] = r == 0 ? sm.cpage[(blk - i0) / kBlocksPerPage] : btab[blk / kBlocksPerPage];
                 } else {
                     us[i0 + pos] = blk;
                 }
@@ -476,11 +485,10 @@ __global__ void __cluster_dims__(kSelCtas, 1, 1) __launch_bounds__(kSelThreads, 
         }
         n_chosen = above + block_reduce_sum(taken_ties, sm.scratch);
     }
-    // blocks this CTA contributes, published in global memory: no CTA reads another's shared memory
-    // after the next barrier, so each may leave as soon as it is done
-    uint32_t *takes = a.takes + (size_t)b * kSelCtas;
-    if (t == 0) takes[c] = consistent ? n_sure + n_chosen : 0u;
-    __syncthreads();   // (the class bytes of the chunk are complete)
+    // blocks this CTA contributes; after reading every CTA's count a CTA only signals the final
+    // barrier, writes its part of the result and then waits there (its shared memory must outlive
+    // the others' reads)
+    if (t == 0) sm.n_take = consistent ? n_sure + n_chosen : 0u;
     cluster.sync();
 
     // ---- 4. ordered output: the sure and chosen blocks of the chunk at the chunk's offset
@@ -488,13 +496,14 @@ __global__ void __cluster_dims__(kSelCtas, 1, 1) __launch_bounds__(kSelThreads, 
     {
         uint32_t tk[kSelCtas];
 #pragma unroll
-        for (int r = 0; r < kSelCtas; ++r) tk[r] = __ldcg(takes + r);
+        for (int r = 0; r < kSelCtas; ++r) tk[r] = *cluster.map_shared_rank(&sm.n_take, r);
 #pragma unroll
         for (int r = 0; r < kSelCtas; ++r) {
             cbase += r < c ? tk[r] : 0u;
             all += tk[r];
         }
     }
+    cluster_arrive_relaxed();
     if (consistent) {
         uint32_t pos = cbase;
         for (int r = 0; r < rounds; ++r) {
@@ -525,11 +534,12 @@ __global__ void __cluster_dims__(kSelCtas, 1, 1) __launch_bounds__(kSelThreads, 
         a.out_count[b] = consistent ? a.k : 0;
         if (consistent && all != (uint32_t)a.k) report(a.ws, CSA_ERR_DEVICE_DATA, (long long)b);
     }
+    cluster_wait();
 }
 
 cudaError_t launch_select(const float *lo, const float *hi, int lstride, const csa_batch &bt, int k,
                           const uint32_t *hist, uint32_t *hist2, uint8_t *status, int sstride, int32_t *uslice,
-                          uint32_t *okeys, int ustride, uint32_t *takes, const uint8_t *keys, int num_pages,
+                          uint32_t *okeys, int ustride, const uint8_t *keys, int num_pages,
                           const uint16_t *iq, const float *iw, int32_t *out_blocks, int32_t *out_count, void *ws,
                           cudaStream_t st)
 {
@@ -544,7 +554,6 @@ cudaError_t launch_select(const float *lo, const float *hi, int lstride, const c
     a.uslice = uslice;
     a.okeys = okeys;
     a.ustride = ustride;
-    a.takes = takes;
     a.seq_len = bt.seq_len;
     a.max_seq_len = bt.max_seq_len;
     a.block_table = bt.block_table;
