@@ -127,11 +127,12 @@ def source_sha(names):
     return h.hexdigest()[:12]
 
 
-KERNEL_SOURCES = {"indexer_full": ["screen.cu", "indexer.cu", "radix.cuh", "common.cuh", "convert.cuh", "pipeline.cuh",
-                                   "tcgen05.cuh"],
-                  "indexer_reindex": ["indexer.cu", "radix.cuh", "common.cuh", "convert.cuh", "pipeline.cuh"],
+KERNEL_SOURCES = {"indexer_full": ["screen.cu", "select.cu", "score.cuh", "radix.cuh", "common.cuh", "convert.cuh",
+                                   "pipeline.cuh", "tcgen05.cuh"],
+                  "indexer_reindex": ["indexer.cu", "score.cuh", "radix.cuh", "common.cuh", "convert.cuh",
+                                      "pipeline.cuh"],
                   "sparse_decode_attn": ["attention_cc.cu", "attention_tc.cu", "attention_common.cuh", "tcgen05.cuh",
-                                         "common.cuh", "convert.cuh"],
+                                         "common.cuh", "convert.cuh", "pipeline.cuh"],
                   "kv_pack_fp4": ["pack.cu", "common.cuh", "convert.cuh"]}
 
 
