@@ -163,8 +163,8 @@ __global__ void __launch_bounds__(256) qterm_kernel(const uint16_t *__restrict__
 }
 
 // ------------------------------------------------------------------------------------------------
-// Step 2: screen.  Persistent CTAs (one per SM), each taking a contiguous range of 128-position
-// tiles (two pages).  Warp 0 resolves tiles 32 at a time (one per lane) and issues the TMA loads of
+// Step 2: screen.  Persistent CTAs (one per SM), each taking every grid-th 128-position tile (two
+// pages) of the batch.  Warp 0 resolves tiles 32 at a time (one per lane) and issues the TMA loads of
 // their two key pages plus, when the sequence changed since that stage's last use, the query-term
 // image.  As soon as a stage lands, warp 1 issues the four K=32 MMAs of its tile into one of six
 // 32-column TMEM accumulators and one of two row-max groups (warps 2-5, 6-9; thread = row) writes
@@ -182,7 +182,6 @@ struct ScreenArgs {
     int num_pages;
     int tiles_per_seq;
     long long total;      // B * tiles_per_seq
-    long long per_cta;    // tiles per CTA
     const float *iw;
     const uint8_t *qt;
     const QMeta *qm;
@@ -276,11 +275,13 @@ __global__ void __launch_bounds__(kScrThreads, 1) screen_kernel(const __grid_con
     extern __shared__ uint8_t scr_raw[];
     ScrSmem &sm = *reinterpret_cast<ScrSmem *>((reinterpret_cast<uintptr_t>(scr_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long first = (long long)blockIdx.x * a.per_cta;
-    const long long last = first + a.per_cta < a.total ? first + a.per_cta : a.total;
+    // CTA c takes tiles c, c + grid, c + 2 grid, ... of the batch's (sequence, tile) slots, so that the
+    // real tiles (slots below each sequence's own length) spread evenly over the CTAs whatever the mix
+    // of lengths; consecutive tiles of a CTA still mostly share a sequence
+    const long long first = blockIdx.x, step = gridDim.x;
     // local tile counters are 32-bit (at most 2^31 tiles per CTA): stage and phase arithmetic by
     // constants then stays a few instructions
-    const uint32_t n_items = last > first ? (uint32_t)(last - first) : 0u;
+    const uint32_t n_items = a.total > first ? (uint32_t)((a.total - first + step - 1) / step) : 0u;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kScrStages; ++s) {
@@ -311,7 +312,7 @@ __global__ void __launch_bounds__(kScrThreads, 1) screen_kernel(const __grid_con
             const uint32_t k = k0 + lane;
             ScrItem it{-1, 0, 0, -1, -1};
             if (k < n_items) {
-                const long long item = first + k;
+                const long long item = first + (long long)k * step;
                 const int b = (int)(item / a.tiles_per_seq), tile = (int)(item % a.tiles_per_seq);
                 const int L = a.seq_len[b];
                 it.b = b;
@@ -602,7 +603,6 @@ cudaError_t launch_screen_bounds(const uint8_t *keys, int num_pages, const csa_b
     sa.tiles_per_seq = (bt.max_seq_len + kScrRows - 1) / kScrRows;
     sa.total = (long long)bt.B * sa.tiles_per_seq;
     const int grid = (int)(sa.total < sm_count() ? sa.total : sm_count());
-    sa.per_cta = (sa.total + grid - 1) / grid;
     sa.iw = iw;
     sa.qt = qt;
     sa.qm = reinterpret_cast<const QMeta *>(qm);
