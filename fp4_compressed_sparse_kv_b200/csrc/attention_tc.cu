@@ -477,17 +477,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_split_tc_kernel(AttnArgs a
             // producers have written half-tile qk, so that the chains of the even and of the odd
             // half-tiles overlap.  (QK(t) precedes PV(t) through the softmax; QK(t+2) follows PV(t)
             // through the producers, who wait for it before reusing the buffer.)  The waits are
-            // polled together, under the same limit as every other wait.
+            // polled together with non-blocking tests (a suspended test of one could miss the other's
+            // completion), under the same limit as every other wait.
             int qk = 0, pv = 0;
             unsigned long long t0 = 0;
             for (uint32_t it = 0; ok && pv < nh; ++it) {
-                if (pv < qk && mbar_try_wait(&ms.p_full[pv & 1], (pv >> 1) & 1)) {
+                if (pv < qk && mbar_test_wait(&ms.p_full[pv & 1], (pv >> 1) & 1)) {
                     tc_fence_after();
                     issue_pv(pv++);
                     t0 = 0;
                     continue;
                 }
-                if (qk < nh && mbar_try_wait(&ms.v_ready[qk & 1], (qk >> 1) & 1)) {
+                if (qk < nh && mbar_test_wait(&ms.v_ready[qk & 1], (qk >> 1) & 1)) {
                     tc_fence_after();
                     issue_qk(qk++);
                     t0 = 0;
