@@ -133,7 +133,8 @@ KERNEL_SOURCES = {"indexer_full": ["screen.cu", "select.cu", "score.cuh", "radix
                                       "pipeline.cuh"],
                   "sparse_decode_attn": ["attention_cc.cu", "attention_tc.cu", "attention_common.cuh", "tcgen05.cuh",
                                          "common.cuh", "convert.cuh", "pipeline.cuh"],
-                  "kv_pack_fp4": ["pack.cu", "common.cuh", "convert.cuh"]}
+                  "kv_pack_fp4": ["pack.cu", "common.cuh", "convert.cuh"],
+                  "kv_pack_fp4_prefill": ["pack.cu", "common.cuh", "convert.cuh"]}
 
 
 def traffic_from_profiles(call, workload):
@@ -168,11 +169,41 @@ def rank_workload(name, rank):
     return w
 
 
-def make_plan(st):
+class Prefill:
+    """The mixed serving step's prefill chunk: w.prefill_tokens new tokens of one sequence, packed into
+    the spare pages, its last 128 tokens into the spare window row (device inputs plus pinned copies)."""
+
+    def __init__(self, st, dev):
+        import numpy as np
+        import torch
+
+        from fp4_compressed_sparse_kv_b200 import synth
+        w = st.w
+        n = w.prefill_tokens
+        rng = synth.rng_for(w, 0, 5000)
+        lat = synth.latents(rng, np.arange(n))
+        key = synth.index_keys(rng, n)
+        spare_row = int(np.setdiff1d(np.arange(st.num_rows), st.swa_row_np)[0])
+        slots = st.prefill_pages[np.arange(n) // 64].astype(np.int64) * 64 + np.arange(n) % 64
+        sw = np.where(np.arange(n) >= n - 128, spare_row * 128 + np.arange(n) % 128, -1).astype(np.int32)
+        self.n = n
+        self.h_lat = torch.from_numpy(lat).view(torch.bfloat16).pin_memory()
+        self.h_key = torch.from_numpy(key).view(torch.bfloat16).pin_memory()
+        self.lat = self.h_lat.to(dev)
+        self.key = self.h_key.to(dev)
+        self.slots = torch.from_numpy(slots).to(dev)
+        self.sw = torch.from_numpy(sw).to(dev)
+
+
+def make_plan(st, prefill=None):
     """The step as a list of (call name, kernels launched, fn): the library's public calls."""
     from fp4_compressed_sparse_kv_b200 import csa
     w = st.w
     plan = []
+    if prefill is not None:
+        plan.append(("kv_pack_fp4_prefill", 1,
+                     lambda: csa.kv_pack_fp4(st.layers[0], prefill.lat, prefill.key, prefill.slots, prefill.sw,
+                                             st.ws)))
     for l, m in enumerate(w.modes):
         f = st.kv_of[l]
         lay = st.layers[f]
@@ -200,7 +231,7 @@ def make_plan(st):
     return plan
 
 
-def algorithmic_bytes(st):
+def algorithmic_bytes(st, prefill=None):
     """Bytes each call must move per step, from the sizes and the selected sets (after a step)."""
     import numpy as np
     w = st.w
@@ -212,6 +243,8 @@ def algorithmic_bytes(st):
     def add(k, v):
         out[k] = out.get(k, 0.0) + float(v)
 
+    if prefill is not None:   # bf16 latent and key in; codes, scales, keys out; 128 window entries
+        add("kv_pack_fp4_prefill", prefill.n * (1024 + 256 + 256 + 32 + 128 + 8 + 4) + 128 * 516)
     for l, m in enumerate(w.modes):
         if m == 0:
             add("kv_pack_fp4", B * (1024 + 256 + 256 + 32 + 128 + 512 + 4 + 12))
@@ -315,7 +348,8 @@ def run_ours(args, rank, world, local):
     t0 = time.time()
     st = workloads.DecodeState(w, device=dev)
     setup_s = time.time() - t0
-    plan = make_plan(st)
+    prefill = Prefill(st, dev) if w.prefill_tokens else None
+    plan = make_plan(st, prefill)
     # L2 flush before every timed step: write 256 MB, then read another 256 MB, so that no input is
     # served from L2 and the L2 holds no dirty lines whose write-back would share DRAM with the step
     flush_w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -335,7 +369,7 @@ def run_ours(args, rank, world, local):
         step()
     torch.cuda.synchronize()
     st.check()
-    bytes_per_call = algorithmic_bytes(st)
+    bytes_per_call = algorithmic_bytes(st, prefill)
     flops_attn = attn_flops(st)
 
     K = args.steps
@@ -405,10 +439,14 @@ def run_ours(args, rank, world, local):
     h_iw = [x.cpu().pin_memory() for x in st.iw]
     h_out = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in st.out]
     h_lse = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in st.lse]
-    h2d = sum(x.numel() * x.element_size() for x in h_lat + h_key + h_q + h_iq + h_iw)
+    h_pre = [prefill.h_lat, prefill.h_key] if prefill is not None else []
+    h2d = sum(x.numel() * x.element_size() for x in h_lat + h_key + h_q + h_iq + h_iw + h_pre)
     d2h = sum(x.numel() * x.element_size() for x in h_out + h_lse)
 
     def e2e_step():
+        if prefill is not None:
+            prefill.lat.copy_(prefill.h_lat, non_blocking=True)
+            prefill.key.copy_(prefill.h_key, non_blocking=True)
         for f in range(n_kv):
             st.new_tokens[f][0].copy_(h_lat[f], non_blocking=True)
             st.new_tokens[f][1].copy_(h_key[f], non_blocking=True)
