@@ -5,10 +5,12 @@
 // main KV is FP4 while the more quantisation-sensitive SWA KV stays FP8.  ailily.cc article
 // "每个 token 只占 890 字节", section 二: one E4M3 scale per 16 channels holds the value range.
 //
-// One warp per token.  Lane g owns 16-channel group g of the 512-channel latent, which is exactly
-// one E4M3 scale: its amax needs no cross-lane step, and its 16 codes are one 8-byte store.  The
-// window entry needs the token's amax, a 5-step warp max.  Loads are 2 x 16 B per lane (latent) and
-// 8 B per lane (key), all coalesced; HBM-bound streaming.
+// One warp per token at a time; for long calls, four consecutive tokens per warp with all their loads
+// issued first.
+// Lane g owns 16-channel group g of the 512-channel latent, which is exactly one E4M3 scale: its amax
+// needs no cross-lane step, and its 16 codes are one 8-byte store.  The window entry needs the
+// token's amax, a 5-step warp max.  Loads are 2 x 16 B per lane (latent) and 8 B per lane (key), all
+// coalesced; HBM-bound streaming.
 //
 // The norm variant starts from the pre-norm latent (ailily.cc article, section 三: the KV latent is
 // RMS-normalised, with weights of magnitude about 1, and rotated by RoPE, which keeps its norm): in
@@ -23,28 +25,26 @@
 
 namespace csa {
 
-template <bool kNorm>
-__global__ void __launch_bounds__(256) kv_pack_kernel(csa_kv_layer layer, const uint16_t *__restrict__ latent,
-                                                      const uint16_t *__restrict__ idx_key,
-                                                      const int64_t *__restrict__ slot,
-                                                      const int32_t *__restrict__ swa_slot, int n, void *ws,
-                                                      const float *__restrict__ norm_w,
-                                                      const float *__restrict__ rope_cs)
-{
-    const int tok = blockIdx.x * 8 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (tok >= n) return;
+// A token's inputs, loaded ahead of its arithmetic.
+struct PackIn {
+    uint4 a, b;     // latent channels 16 lane .. 16 lane + 15 (bf16)
+    uint2 kw;       // indexer-key channels 4 lane .. 4 lane + 3 (bf16)
+    int64_t s;      // main slot
+    int32_t ss;     // window slot
+};
 
-    const int64_t s = slot[tok];
-    const int32_t ss = swa_slot ? swa_slot[tok] : -1;
+template <bool kNorm>
+__device__ __forceinline__ void pack_token(const csa_kv_layer &layer, const PackIn &in, int tok, int lane, void *ws,
+                                           const float *__restrict__ norm_w, const float *__restrict__ rope_cs)
+{
+    const int64_t s = in.s;
+    const int32_t ss = in.ss;
     const bool main_ok = s >= 0 && s < (int64_t)layer.num_pages * kPage;
     const bool swa_ok = ss >= 0 && ss < layer.num_rows * kWindow;
     if (lane == 0 && (!main_ok || (ss >= 0 && !swa_ok))) report(ws, CSA_ERR_DEVICE_DATA, tok);
 
     // 16 channels of group `lane`
-    const uint4 *src = reinterpret_cast<const uint4 *>(latent + (size_t)tok * kLatent) + 2 * lane;
-    const uint4 a = src[0], b = src[1];
-    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    const uint32_t w[8] = {in.a.x, in.a.y, in.a.z, in.a.w, in.b.x, in.b.y, in.b.z, in.b.w};
     float x[16];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -105,7 +105,7 @@ __global__ void __launch_bounds__(256) kv_pack_kernel(csa_kv_layer layer, const 
         layer.scales[s * kScaleBytes + lane] = sc;
 
         // indexer key: channels 4*lane .. 4*lane+3, plain E4M3 cast
-        const uint2 kw = reinterpret_cast<const uint2 *>(idx_key + (size_t)tok * kIdxDim)[lane];
+        const uint2 kw = in.kw;
         const uint32_t k01 = f32x2_to_e4m3x2(bf16_lo(kw.x), bf16_hi(kw.x));
         const uint32_t k23 = f32x2_to_e4m3x2(bf16_lo(kw.y), bf16_hi(kw.y));
         reinterpret_cast<uint32_t *>(layer.keys + s * kIdxDim)[lane] = k01 | (k23 << 16);
@@ -132,12 +132,51 @@ __global__ void __launch_bounds__(256) kv_pack_kernel(csa_kv_layer layer, const 
     }
 }
 
+
+// Each warp packs kTok consecutive tokens: their loads are issued together, then each token's
+// arithmetic runs on registers, so every warp keeps several tokens' bytes in flight (prefill chunks);
+// a decode batch of a few tokens takes one token per warp, its latency being one token's.
+constexpr int kPackTokLarge = 4;
+constexpr int kPackLargeFrom = 4096;   // tokens per call from which warps take kPackTokLarge tokens
+
+template <bool kNorm, int kPackTok>
+__global__ void __launch_bounds__(256) kv_pack_kernel(csa_kv_layer layer, const uint16_t *__restrict__ latent,
+                                                      const uint16_t *__restrict__ idx_key,
+                                                      const int64_t *__restrict__ slot,
+                                                      const int32_t *__restrict__ swa_slot, int n, void *ws,
+                                                      const float *__restrict__ norm_w,
+                                                      const float *__restrict__ rope_cs)
+{
+    const int tok0 = (blockIdx.x * 8 + (threadIdx.x >> 5)) * kPackTok;
+    const int lane = threadIdx.x & 31;
+    PackIn in[kPackTok];
+#pragma unroll
+    for (int i = 0; i < kPackTok; ++i) {
+        const int tok = tok0 + i;
+        if (tok < n) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(latent + (size_t)tok * kLatent) + 2 * lane;
+            in[i].a = src[0];
+            in[i].b = src[1];
+            in[i].kw = reinterpret_cast<const uint2 *>(idx_key + (size_t)tok * kIdxDim)[lane];
+            in[i].s = slot[tok];
+            in[i].ss = swa_slot ? swa_slot[tok] : -1;
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < kPackTok; ++i)
+        if (tok0 + i < n) pack_token<kNorm>(layer, in[i], tok0 + i, lane, ws, norm_w, rope_cs);
+}
+
 cudaError_t launch_kv_pack(const csa_kv_layer &layer, const uint16_t *latent, const uint16_t *idx_key,
                            const int64_t *slot, const int32_t *swa_slot, int n, void *ws, cudaStream_t st)
 {
     if (n == 0) return cudaSuccess;
-    kv_pack_kernel<false><<<(n + 7) / 8, 256, 0, st>>>(layer, latent, idx_key, slot, swa_slot, n, ws, nullptr,
-                                                       nullptr);
+    if (n >= kPackLargeFrom)
+        kv_pack_kernel<false, kPackTokLarge><<<(n + 8 * kPackTokLarge - 1) / (8 * kPackTokLarge), 256, 0, st>>>(
+            layer, latent, idx_key, slot, swa_slot, n, ws, nullptr, nullptr);
+    else
+        kv_pack_kernel<false, 1><<<(n + 7) / 8, 256, 0, st>>>(layer, latent, idx_key, slot, swa_slot, n, ws, nullptr,
+                                                             nullptr);
     return cudaGetLastError();
 }
 
@@ -146,8 +185,12 @@ cudaError_t launch_kv_norm_rope_pack(const csa_kv_layer &layer, const uint16_t *
                                      const int32_t *swa_slot, int n, void *ws, cudaStream_t st)
 {
     if (n == 0) return cudaSuccess;
-    kv_pack_kernel<true><<<(n + 7) / 8, 256, 0, st>>>(layer, latent, idx_key, slot, swa_slot, n, ws, norm_w,
-                                                      rope_cs);
+    if (n >= kPackLargeFrom)
+        kv_pack_kernel<true, kPackTokLarge><<<(n + 8 * kPackTokLarge - 1) / (8 * kPackTokLarge), 256, 0, st>>>(
+            layer, latent, idx_key, slot, swa_slot, n, ws, norm_w, rope_cs);
+    else
+        kv_pack_kernel<true, 1><<<(n + 7) / 8, 256, 0, st>>>(layer, latent, idx_key, slot, swa_slot, n, ws, norm_w,
+                                                            rope_cs);
     return cudaGetLastError();
 }
 

@@ -46,10 +46,10 @@ def assert_same(got, ref, keys):
         assert bad.size == 0, "%s differs in %d tokens, first %s" % (k, bad.size, bad[:5])
 
 
-@pytest.mark.parametrize("heavy", [False, True])
-def test_pack_bit_exact_generated(heavy):
-    rng = np.random.default_rng(60 + heavy)
-    n = 3001
+@pytest.mark.parametrize("heavy,n", [(False, 3001), (True, 3001), (False, 6003)])
+def test_pack_bit_exact_generated(heavy, n):
+    """3,001 tokens take one token per warp; 6,003 (a ragged last warp) four tokens per warp."""
+    rng = np.random.default_rng(60 + heavy + n)
     lat = synth.latents(rng, rng.integers(0, 1 << 20, n), heavy_tail=heavy)
     key = synth.index_keys(rng, n)
     got = run_pack(lat, key)
