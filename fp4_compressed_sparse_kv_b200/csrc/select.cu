@@ -15,11 +15,12 @@
 // block with upper > U has lower > X, and fewer than k blocks do.  If some bound of the sequence is
 // not finite, U is the largest key and no block is sure.
 //
-// One cluster of 8 CTAs per sequence, CTA c owning a contiguous chunk of its blocks (thread t: 8
-// consecutive blocks per round of 2,048).  The cluster's hardware barrier orders the steps; partial
-// results are exchanged through distributed shared memory, the second histogram and the per-CTA
-// result counts through global memory.  Every wait is a cluster barrier, which all 8 CTAs reach on
-// every path (every branch below depends only on per-sequence values), so no wait can be left open.
+// One cluster of 8 CTAs per sequence (16 for batches of up to 18 sequences), CTA c owning a
+// contiguous chunk of its blocks (thread t: 8 consecutive blocks per round of 2,048).  The cluster's
+// hardware barrier orders the steps; partial results are exchanged through distributed shared
+// memory, the second histogram through global memory.  Every wait is a cluster barrier, which all
+// CTAs of the cluster reach on every path (every branch below depends only on per-sequence values),
+// so no wait can be left open.
 //   1. second histogram and the widest interval over the chunk;            barrier
 //   2. T and U; classify the chunk into class bytes, the uncertain blocks listed in block order
 //      with their pages; score them exactly (the binary32 chain of csa.h);  barrier
@@ -39,7 +40,6 @@ namespace cg = cooperative_groups;
 
 namespace csa {
 
-constexpr int kSelCtas = 8;              // CTAs per sequence: one portable-size cluster
 constexpr int kSelThreads = 256;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kSelPer = 8;               // consecutive blocks per thread in one round
@@ -181,7 +181,8 @@ __device__ __forceinline__ void load8(const float *p, int i, int end, float (&v)
     }
 }
 
-__global__ void __cluster_dims__(kSelCtas, 1, 1) __launch_bounds__(kSelThreads, 2) select_kernel(const SelArgs a)
+template <int kSelCtas>
+__global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelArgs a)
 {
     __shared__ SelSmem sm;
     cg::cluster_group cluster = cg::this_cluster();
@@ -566,7 +567,54 @@ cudaError_t launch_select(const float *lo, const float *hi, int lstride, const c
     a.out_blocks = out_blocks;
     a.out_count = out_count;
     a.ws = ws;
-    return launch_overlapped(select_kernel, dim3(kSelCtas, bt.B), dim3(kSelThreads), 0, st, a);
+    // 16-CTA clusters (non-portable) when the batch is small enough for them to fill at most two
+    // CTAs per SM and the device can place one; 8-CTA clusters otherwise
+    static int cap16[64];   // per device: 0 unknown, 1 yes, 2 no
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    int nsm = 0;
+    if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    bool use16 = false;
+    if (bt.B * 16 <= 2 * nsm && dev >= 0 && dev < 64) {
+        if (cap16[dev] == 0) {
+            int ok = 0;
+            if (cudaFuncSetAttribute(select_kernel<16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+                cudaSuccess) {
+                cudaLaunchConfig_t q = {};
+                q.gridDim = dim3(16, 1);
+                q.blockDim = dim3(kSelThreads);
+                cudaLaunchAttribute qa[1];
+                qa[0].id = cudaLaunchAttributeClusterDimension;
+                qa[0].val.clusterDim.x = 16;
+                qa[0].val.clusterDim.y = 1;
+                qa[0].val.clusterDim.z = 1;
+                q.attrs = qa;
+                q.numAttrs = 1;
+                int n = 0;
+                ok = cudaOccupancyMaxActiveClusters(&n, select_kernel<16>, &q) == cudaSuccess && n >= 1;
+            }
+            cudaGetLastError();
+            cap16[dev] = ok ? 1 : 2;
+        }
+        use16 = cap16[dev] == 1;
+    }
+    const int nc = use16 ? 16 : 8;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(nc, bt.B);
+    cfg.blockDim = dim3(kSelThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = nc;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return use16 ? cudaLaunchKernelEx(&cfg, select_kernel<16>, a) : cudaLaunchKernelEx(&cfg, select_kernel<8>, a);
 }
 
 }  // namespace csa
