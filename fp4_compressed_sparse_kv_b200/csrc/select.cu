@@ -538,6 +538,59 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelArgs a)
     cluster_wait();
 }
 
+// Launch kernel16 with 16-CTA clusters (non-portable) when the batch is small enough for them to fill
+// at most two CTAs per SM and the device can place one, kernel8 with 8-CTA clusters otherwise; grid
+// (cluster size, B), programmatic dependent launch.
+template <typename Args>
+cudaError_t launch_clusters(void (*kernel16)(Args), void (*kernel8)(Args), int B, cudaStream_t st, const Args &a)
+{
+    static int cap16[64];   // per device: 0 unknown, 1 yes, 2 no
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    int nsm = 0;
+    if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    bool use16 = false;
+    if (B * 16 <= 2 * nsm && dev >= 0 && dev < 64) {
+        if (cap16[dev] == 0) {   // first use on this device (a race here only repeats the query)
+            int ok = 0;
+            if (cudaFuncSetAttribute(kernel16, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
+                cudaLaunchConfig_t q = {};
+                q.gridDim = dim3(16, 1);
+                q.blockDim = dim3(kSelThreads);
+                cudaLaunchAttribute qa[1];
+                qa[0].id = cudaLaunchAttributeClusterDimension;
+                qa[0].val.clusterDim.x = 16;
+                qa[0].val.clusterDim.y = 1;
+                qa[0].val.clusterDim.z = 1;
+                q.attrs = qa;
+                q.numAttrs = 1;
+                int n = 0;
+                ok = cudaOccupancyMaxActiveClusters(&n, kernel16, &q) == cudaSuccess && n >= 1;
+            }
+            cudaGetLastError();
+            cap16[dev] = ok ? 1 : 2;
+        }
+        use16 = cap16[dev] == 1;
+    }
+    const int nc = use16 ? 16 : 8;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(nc, B);
+    cfg.blockDim = dim3(kSelThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = nc;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return use16 ? cudaLaunchKernelEx(&cfg, kernel16, a) : cudaLaunchKernelEx(&cfg, kernel8, a);
+}
+
 cudaError_t launch_select(const float *lo, const float *hi, int lstride, const csa_batch &bt, int k,
                           const uint32_t *hist, uint32_t *hist2, uint8_t *status, int sstride, int32_t *uslice,
                           uint32_t *okeys, int ustride, const uint8_t *keys, int num_pages,
@@ -567,54 +620,7 @@ cudaError_t launch_select(const float *lo, const float *hi, int lstride, const c
     a.out_blocks = out_blocks;
     a.out_count = out_count;
     a.ws = ws;
-    // 16-CTA clusters (non-portable) when the batch is small enough for them to fill at most two
-    // CTAs per SM and the device can place one; 8-CTA clusters otherwise
-    static int cap16[64];   // per device: 0 unknown, 1 yes, 2 no
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    int nsm = 0;
-    if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    bool use16 = false;
-    if (bt.B * 16 <= 2 * nsm && dev >= 0 && dev < 64) {
-        if (cap16[dev] == 0) {
-            int ok = 0;
-            if (cudaFuncSetAttribute(select_kernel<16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
-                cudaSuccess) {
-                cudaLaunchConfig_t q = {};
-                q.gridDim = dim3(16, 1);
-                q.blockDim = dim3(kSelThreads);
-                cudaLaunchAttribute qa[1];
-                qa[0].id = cudaLaunchAttributeClusterDimension;
-                qa[0].val.clusterDim.x = 16;
-                qa[0].val.clusterDim.y = 1;
-                qa[0].val.clusterDim.z = 1;
-                q.attrs = qa;
-                q.numAttrs = 1;
-                int n = 0;
-                ok = cudaOccupancyMaxActiveClusters(&n, select_kernel<16>, &q) == cudaSuccess && n >= 1;
-            }
-            cudaGetLastError();
-            cap16[dev] = ok ? 1 : 2;
-        }
-        use16 = cap16[dev] == 1;
-    }
-    const int nc = use16 ? 16 : 8;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(nc, bt.B);
-    cfg.blockDim = dim3(kSelThreads);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = nc;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 2;
-    return use16 ? cudaLaunchKernelEx(&cfg, select_kernel<16>, a) : cudaLaunchKernelEx(&cfg, select_kernel<8>, a);
+    return launch_clusters(select_kernel<16>, select_kernel<8>, bt.B, st, a);
 }
 
 }  // namespace csa
