@@ -90,7 +90,11 @@ __global__ void __launch_bounds__(256) qterm_kernel(const uint16_t *__restrict__
                                                     uint32_t *__restrict__ hist, uint32_t *__restrict__ hist2)
 {
     const int b = blockIdx.x, h = threadIdx.x >> 5, l = threadIdx.x & 31;
-    grid_dep_launch();   // the screen may start streaming keys meanwhile
+    // launched so that it may be scheduled while the stream's previous kernel (e.g. the pack of the
+    // new tokens, whose keys the screen reads) finishes: wait for it, then let the screen start
+    // streaming keys while the query terms are formed
+    grid_dep_wait();
+    grid_dep_launch();
     // the histograms the later steps accumulate into start from zero on every call
     for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) {
         hist[(size_t)b * kHistBins + i] = 0u;
@@ -590,8 +594,9 @@ cudaError_t launch_screen_bounds(const uint8_t *keys, int num_pages, const csa_b
     CUtensorMap map;
     if ((e = keys_tensor_map(keys, num_pages, &map)) != cudaSuccess) return e;
 
-    qterm_kernel<<<bt.B, 256, 0, st>>>(iq, iw, qt, reinterpret_cast<QMeta *>(qm), hist, hist2);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_overlapped(qterm_kernel, dim3(bt.B), dim3(256), 0, st, iq, iw, qt, reinterpret_cast<QMeta *>(qm),
+                               hist, hist2)) != cudaSuccess)
+        return e;
 
     ScreenArgs sa;
     sa.seq_len = bt.seq_len;

@@ -28,6 +28,8 @@
 //      each CTA marking its own: ranked by counting against the whole list when there are few, else
 //      radix-selected over the cluster;                                    barrier
 //   4. the sure and chosen blocks of each chunk written in ascending order at the chunk's offset.
+#include <atomic>
+
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -544,7 +546,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SelArgs a)
 template <typename Args>
 cudaError_t launch_clusters(void (*kernel16)(Args), void (*kernel8)(Args), int B, cudaStream_t st, const Args &a)
 {
-    static int cap16[64];   // per device: 0 unknown, 1 yes, 2 no
+    static std::atomic<int> cap16[64];   // per device: 0 unknown, 1 yes, 2 no
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -552,7 +554,7 @@ cudaError_t launch_clusters(void (*kernel16)(Args), void (*kernel8)(Args), int B
     if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     bool use16 = false;
     if (B * 16 <= 2 * nsm && dev >= 0 && dev < 64) {
-        if (cap16[dev] == 0) {   // first use on this device (a race here only repeats the query)
+        if (cap16[dev].load() == 0) {   // first use on this device (concurrent callers may both query)
             int ok = 0;
             if (cudaFuncSetAttribute(kernel16, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess) {
                 cudaLaunchConfig_t q = {};
@@ -569,9 +571,9 @@ cudaError_t launch_clusters(void (*kernel16)(Args), void (*kernel8)(Args), int B
                 ok = cudaOccupancyMaxActiveClusters(&n, kernel16, &q) == cudaSuccess && n >= 1;
             }
             cudaGetLastError();
-            cap16[dev] = ok ? 1 : 2;
+            cap16[dev].store(ok ? 1 : 2);
         }
-        use16 = cap16[dev] == 1;
+        use16 = cap16[dev].load() == 1;
     }
     const int nc = use16 ? 16 : 8;
     cudaLaunchConfig_t cfg = {};
