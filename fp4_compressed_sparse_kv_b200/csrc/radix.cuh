@@ -52,6 +52,30 @@ __device__ __forceinline__ uint32_t block_reduce_sum(uint32_t v, uint32_t *scrat
     return v;
 }
 
+// Exclusive prefix of v over the CTA in thread order (blockDim.x a multiple of 32, at most 1024
+// threads; scratch holds at least 32 words); every thread also gets the total.  Two barriers.
+__device__ __forceinline__ uint32_t cta_scan(uint32_t v, uint32_t *scratch, uint32_t &total)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (int)(blockDim.x >> 5);
+    uint32_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) scratch[warp] = x;
+    __syncthreads();
+    uint32_t before = 0;
+    total = 0;
+    for (int w = 0; w < nw; ++w) {
+        const uint32_t c = scratch[w];
+        before += w < warp ? c : 0u;
+        total += c;
+    }
+    __syncthreads();
+    return before + x - v;
+}
+
 // The k-th largest of n keys (1 <= k <= n), MSB first in digits of up to 8 bits with per-warp
 // shared-memory histograms (whist: kWarps x 256 words).  The bits every key shares (the common
 // prefix of the smallest and largest key) are skipped.  Bits below stop_bit may stay unresolved:

@@ -94,30 +94,6 @@ struct SelSmem {
     uint32_t sel[2];
 };
 
-// Exclusive prefix of v over the CTA in thread order; every thread also gets the total.  Two barriers.
-__device__ __forceinline__ uint32_t cta_scan(uint32_t v, uint32_t *scratch, uint32_t &total)
-{
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    uint32_t x = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) scratch[warp] = x;
-    __syncthreads();
-    uint32_t before = 0;
-    total = 0;
-#pragma unroll
-    for (int w = 0; w < kSelWarps; ++w) {
-        const uint32_t c = scratch[w];
-        before += w < warp ? c : 0u;
-        total += c;
-    }
-    __syncthreads();
-    return before + x - v;
-}
-
 // Over a kHistBins-bin histogram h (read from L2: other CTAs of the cluster add to it): the bin
 // holding the rank-th largest element (1-based) and that element's rank inside the bin; every
 // thread gets both.  If the counts fall short of rank: bin 0 (a threshold that keeps everything).
