@@ -59,7 +59,15 @@ def measured_peaks():
         return dict(hbm_gbs=float(d["hbm_gbs"]), bf16_tflops=float(d["bf16_tflops"]),
                     bf16_tflops_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
                     source="measured")
+    # an earlier B200 measurement (STREAM-style copy; cuBLAS bf16 GEMM burst and sustained), used only
+    # when no measured-peaks file is present
     return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def peak_label(peaks, key, note=""):
+    if peaks["source"] == "measured":
+        return "measured (MEASURED_PEAKS.json %s%s)" % (key, note)
+    return "fallback (no MEASURED_PEAKS.json; earlier B200 measurement of %s%s)" % (key, note)
 
 
 # ------------------------------------------------------------------------------------------------
@@ -542,13 +550,13 @@ def run_ours(args, rank, world, local):
         achieved = per_launch_flops / (per_launch_ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "kernel": dominant, "achieved": round(achieved, 1), "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": traffic,
-                "peak_source": peaks["source"] + " (MEASURED_PEAKS.json bf16_tflops, burst; f16 same rate)",
+                "peak_source": peak_label(peaks, "bf16_tflops", ", burst; f16 same rate"),
                 "bytes_frac": round(per_launch_bytes / (per_launch_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
     else:
         achieved = per_launch_bytes / (per_launch_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "kernel": dominant, "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": traffic, "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs)"}
+                "traffic": traffic, "peak_source": peak_label(peaks, "hbm_gbs")}
     step_bytes = sum(bytes_per_call.values())
     attn_ms = call_ms.get("sparse_decode_attn", 0.0)
     line = {
