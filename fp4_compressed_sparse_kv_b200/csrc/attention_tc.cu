@@ -295,6 +295,63 @@ __device__ __forceinline__ void tc_st16_u(uint32_t taddr, const uint32_t *v)
         : "memory");
 }
 
+// 32 lanes x 8 consecutive 32-bit columns (thread i: lane i), waited for in the same statement; and
+// the matching store.
+__device__ __forceinline__ void tc_ld8_sync(uint32_t taddr, float *v)
+{
+    uint32_t r[8];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tc_st8(uint32_t taddr, const float *v)
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+                 "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+                 "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+                 "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7]))
+                 : "memory");
+}
+
+// Two loads of 16 lanes x 16 columns with a half-warp split: thread i < 16 gets lane base+i, columns
+// [col, col+16) and thread i >= 16 lane base+i-16, columns [col+32, col+48), from each address; one
+// wait for both in the same statement.
+__device__ __forceinline__ void tc_ld16x32bx2_x16_pair(uint32_t ta, uint32_t tb, float *a, float *b)
+{
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%32], 32;\n"
+        "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 "
+        "{%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%33], 32;\n"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(ta), "r"(tb)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        a[i] = __uint_as_float(r[i]);
+        b[i] = __uint_as_float(r[16 + i]);
+    }
+}
+
+// One arrival per warp: every lane's earlier writes (and its proxy or tcgen05 fences) are ordered
+// before lane 0's arrive by the warp barrier.  Barriers that warps arrive on count warps.
+__device__ __forceinline__ void warp_arrive(uint64_t *bar)
+{
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
 // Q of heads h0..h0+63 into TMEM as the A operand of the QK MMAs, scaled by one power of two 2^k that
 // puts the largest |q| of the 64 heads in [2^13, 2^14); returns tau * log2(e) * 2^-k, the factor that
 // turns an accumulated score into the log2 domain (every thread gets it).  Warp w < 16 writes TMEM
@@ -349,7 +406,7 @@ __device__ __forceinline__ float load_q(const AttnArgs &a, TcMisc &ms, uint32_t 
         }
         tc_wait_st();
         tc_fence_before();
-        mbar_arrive(&ms.q_ready);
+        warp_arrive(&ms.q_ready);
     }
     return a.sm_scale * exp2f((float)-k) * kLog2e;
 }
@@ -369,16 +426,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_split_tc_kernel(AttnArgs a
     const int h0 = hg * kTcHeads;
 
     if (threadIdx.x == 0) {
-        mbar_init(&ms.q_ready, 512);   // the Q-loading warps 0-15
+        mbar_init(&ms.q_ready, 16);    // the Q-loading warps 0-15
         mbar_init(&ms.o_done, 2);
         for (int i = 0; i < kStages; ++i) {
-            mbar_init(&ms.v_ready[i], kProducers);
+            mbar_init(&ms.v_ready[i], kProducers / 32);
             mbar_init(&ms.v_free[i], 2);
-            mbar_init(&ms.p_full[i], kSoftmax);
+            mbar_init(&ms.p_full[i], kSoftmax / 32);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&ms.s_full[i], 2);
-            mbar_init(&ms.s_free[i], kSoftmax);
+            mbar_init(&ms.s_free[i], kSoftmax / 32);
         }
         for (int r = 0; r < 4; ++r) mbar_init(&ms.final_bar[r], 1);
         ms.abort_flag = 0;
@@ -394,6 +451,119 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_split_tc_kernel(AttnArgs a
     const uint32_t tmem = ms.tmem_base;
     // Q is an input of the step, not a result of the previous grid: load it while that grid finishes
     const float zs = load_q(a, ms, tmem, b, h0, threadIdx.x);
+    bool ok = true;
+
+    // One tile of the softmax (warps 16-19): scores of tile t from TMEM, the running maxima (O^T
+    // rescaled when one grows by more than 2^8), P^T into the tile's P buffer.  A dry call (before
+    // the previous grid has finished) runs the same code on whatever the S and O^T columns hold,
+    // with no waits or arrivals and the rescale forced, so that the first real tile runs warm; it
+    // writes only the P buffer of tile 2, O^T and the rescale factors, all rewritten before use.
+    const int q = warp - kSoftmaxWarp;       // TMEM quarter: heads 16q .. 16q+15
+    const int u = lane >> 4;                 // this thread's entries 32u .. 32u+31 of a tile
+    const int hl = 16 * q + (lane & 15);     // this thread's head
+    const uint32_t tq = tmem + ((uint32_t)((32 * q) & 127) << 16);
+    auto softmax_tile = [&](int t, bool dry, float &m_run, float &lsum) {
+        const int p = dry ? 2 : t % kStages, sb = dry ? 0 : t & 1;
+        // v_ready: the producers' valid-row mask of this tile; s_full: both halves of its scores
+        if (!dry)
+            ok = bar_and(1, kSoftmax, ok && warp_wait(&ms.v_ready[p], (uint32_t)(t / kStages) & 1u, &ms.abort_flag, a.ws, 9) &&
+                                          warp_wait(&ms.s_full[sb], (uint32_t)(t >> 1) & 1u, &ms.abort_flag, a.ws, 6));
+        if (ok) {
+            tc_fence_after();
+            // z[j] = S_0 + S_1 of entry 32u + j of head hl (unscaled): 16-lane loads whose first
+            // half-warp reads columns c.. and second half-warp columns c + 32.. of the same lanes
+            float z[32];
+#pragma unroll
+            for (int pc = 0; pc < 2; ++pc) {
+                float s0[16], s1[16];
+                tc_ld16x32bx2_x16_pair(tq + kColS + 64 * sb + 16 * pc, tq + (16u << 16) + kColS + 64 * sb + 16 * pc,
+                                       s0, s1);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) z[16 * pc + i] = s0[i] + s1[i];
+            }
+            tc_fence_before();
+            if (!dry) warp_arrive(&ms.s_free[sb]);   // QK of tile t + 2 may overwrite these columns
+            const uint32_t vbits = dry ? 0xFFFFFFFFu : (uint32_t)(ms.vmask[p] >> (32 * u));
+            if (vbits != 0xFFFFFFFFu) {
+                // a tile with masked entries (the sequence's last): their scores drop out
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (!((vbits >> i) & 1u)) z[i] = -INFINITY;
+            }
+            float mt = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) mt = fmaxf(mt, z[i]);
+            // the head's maximum over the tile, log2 domain (zs > 0: the scaled maximum is the
+            // maximum of the scaled scores)
+            mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16)) * zs;
+            const bool need = dry || mt > m_run + kLazy;
+            if (bar_or(1, kSoftmax, need)) {
+                // some head's maximum grew: new maxima, and O^T rescaled column by column
+                const float mn = need ? fmaxf(m_run, mt) : m_run;
+                const float al = exp2f(m_run - mn);   // 0 while m_run is kNoMax, 1 if unchanged
+                if (u == 0) ms.alpha[hl] = al;
+                lsum *= al;
+                m_run = mn;
+                bar_sync(1, kSoftmax);   // every head's factor visible
+                if (t > 0 || dry) {
+                    // this warp's lanes of the four O^T M-tiles, once PV(t-1) has completed
+                    const int tp = t - 1;
+                    const bool pv_ok = dry || warp_wait(&ms.v_free[tp % kStages], (uint32_t)(tp / kStages) & 1u,
+                                                        &ms.abort_flag, a.ws, 7);
+                    if (pv_ok) {
+                        tc_fence_after();
+#pragma unroll 1
+                        for (int k = 0; k < 32; ++k) {
+                            float o[8];
+                            const uint32_t col = kColO + 8 * k;   // M-tile k/8, heads 8(k%8) ..
+                            tc_ld8_sync(tq + col, o);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) o[i] *= ms.alpha[8 * (k & 7) + i];
+                            tc_st8(tq + col, o);
+                        }
+                        tc_wait_st();
+                    }
+                    ok = pv_ok;
+                }
+            }
+            // P^T row hl, entries 32u .. 32u+31: four 16-byte units of the 128-byte swizzled row;
+            // p = 2^(z zs - m + 7), 0 for a masked entry (z = -inf)
+            const float mref = m_run - kPOffset;
+            float ls = 0.f;
+            uint8_t *Pb = P + p * kPBuf;
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                uint32_t pk[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float p0 = exp2f(fmaf(z[8 * g + 2 * i], zs, -mref));
+                    const float p1 = exp2f(fmaf(z[8 * g + 2 * i + 1], zs, -mref));
+                    ls += p0 + p1;
+                    pk[i] = pack_f16x2(p0, p1);
+                }
+                *reinterpret_cast<uint4 *>(Pb + swz((uint32_t)hl, (uint32_t)(4 * u + g))) =
+                    make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+            lsum += ls;
+            fence_async_smem();
+            tc_fence_before();
+        } else if (!dry) {
+            warp_arrive(&ms.s_free[sb]);
+        }
+        if (!dry) warp_arrive(&ms.p_full[p]);
+    };
+
+    // warm the first-pass code of the softmax and of the producers while the previous grid finishes
+    if (warp >= kSoftmaxWarp && warp < kIssuerWarp) {
+        float dm = kNoMax, dl = 0.f;
+        softmax_tile(0, true, dm, dl);
+    } else if (warp < kSoftmaxWarp) {
+        RawHalf dummy;
+        dummy.row = 0;
+        dummy.code[0] = dummy.code[1] = make_uint4(0u, 0u, 0u, 0u);
+        dummy.sc = 0x38383838u;   // E4M3 1.0
+        dummy.write(a, V + 2 * kVBuf, threadIdx.x & (kHalf - 1), threadIdx.x >> 6);
+    }
     grid_dep_wait();   // the selected blocks of the previous grid
 
     if (threadIdx.x == 0) {
@@ -424,7 +594,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_split_tc_kernel(AttnArgs a
         return;
     }
 
-    bool ok = true;
     if (warp >= kIssuerWarp) {
         // ------------------------------- MMA issuers -------------------------------
         const int r = warp - kIssuerWarp;
@@ -496,7 +665,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_split_tc_kernel(AttnArgs a
                 if (lane == 0) reinterpret_cast<volatile uint32_t *>(&ms.vmask[p])[warp] = vb;
             }
             fence_async_smem();
-            mbar_arrive(&ms.v_ready[p]);
+            warp_arrive(&ms.v_ready[p]);
             if (t + 2 < nh) {
                 if ((t + 2) % kTabHalves == 0) {
                     // the next tiles' entry addresses (every producer has fetched from the old ones)
@@ -514,97 +683,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_split_tc_kernel(AttnArgs a
         }
     } else {
         // ------------------------------- softmax -------------------------------
-        const int q = warp - kSoftmaxWarp;       // TMEM quarter: heads 16q .. 16q+15
-        const int u = lane >> 4;                 // this thread's entries 32u .. 32u+31 of a tile
-        const int hl = 16 * q + (lane & 15);     // this thread's head
-        const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16);
         float m_run = kNoMax;                    // the head's running maximum (log2 domain), as the partner has it
         float lsum = 0.f;                        // this thread's share of the head's denominator
-        for (int t = 0; t < nh; ++t) {
-            const int p = t % kStages, sb = t & 1;
-            // v_ready: the producers' valid-row mask of this tile; s_full: both halves of its scores
-            ok = bar_and(1, kSoftmax, ok && warp_wait(&ms.v_ready[p], (uint32_t)(t / kStages) & 1u, &ms.abort_flag, a.ws, 9) &&
-                                          warp_wait(&ms.s_full[sb], (uint32_t)(t >> 1) & 1u, &ms.abort_flag, a.ws, 6));
-            if (ok) {
-                tc_fence_after();
-                // z[j] = S_0 + S_1 of entry 32u + j: this lane holds S_u of all 64 entries of head hl,
-                // lane ^ 16 the other half
-                float z[32];
-#pragma unroll
-                for (int pc = 0; pc < 4; ++pc) {
-                    // columns 16pc .. 16pc+15: entries of this thread when pc / 2 == u
-                    float r[16];
-                    tc_ld16_sync(tq + kColS + 64 * sb + 16 * pc, r);
-                    const bool mine = (pc >> 1) == u;
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float o = __shfl_xor_sync(0xffffffffu, r[i], 16);
-                        if (mine) z[16 * (pc & 1) + i] = r[i] + o;
-                    }
-                }
-                tc_fence_before();
-                mbar_arrive(&ms.s_free[sb]);   // QK of tile t + 2 may overwrite these columns
-                const uint32_t vbits = (uint32_t)(ms.vmask[p] >> (32 * u));
-                float mt = -INFINITY;
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    z[i] = ((vbits >> i) & 1u) ? z[i] * zs : -INFINITY;
-                    mt = fmaxf(mt, z[i]);
-                }
-                mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));   // the head's maximum over the tile
-                const bool need = mt > m_run + kLazy;
-                if (bar_or(1, kSoftmax, need)) {
-                    // some head's maximum grew: new maxima, and O^T rescaled column by column
-                    const float mn = need ? fmaxf(m_run, mt) : m_run;
-                    const float al = exp2f(m_run - mn);   // 0 while m_run is kNoMax, 1 if unchanged
-                    if (u == 0) ms.alpha[hl] = al;
-                    lsum *= al;
-                    m_run = mn;
-                    bar_sync(1, kSoftmax);   // every head's factor visible
-                    if (t > 0) {
-                        // this warp's lanes of the four O^T M-tiles, once PV(t-1) has completed
-                        const int tp = t - 1;
-                        const bool pv_ok = warp_wait(&ms.v_free[tp % kStages], (uint32_t)(tp / kStages) & 1u,
-                                                     &ms.abort_flag, a.ws, 7);
-                        if (pv_ok) {
-                            tc_fence_after();
-#pragma unroll 1
-                            for (int k = 0; k < 16; ++k) {
-                                float o[16];
-                                const uint32_t col = kColO + 16 * k;   // M-tile k/4, heads 16(k%4) ..
-                                tc_ld16_sync(tq + col, o);
-#pragma unroll
-                                for (int i = 0; i < 16; ++i) o[i] *= ms.alpha[16 * (k & 3) + i];
-                                tc_st16(tq + col, o);
-                            }
-                            tc_wait_st();
-                        }
-                        ok = pv_ok;
-                    }
-                }
-                // P^T row hl, entries 32u .. 32u+31: four 16-byte units of the 128-byte swizzled row
-                const float mref = m_run - kPOffset;
-                uint32_t pk[16];
-                float ls = 0.f;
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float p0 = exp2f(z[2 * i] - mref), p1 = exp2f(z[2 * i + 1] - mref);
-                    ls += p0 + p1;
-                    pk[i] = pack_f16x2(p0, p1);
-                }
-                lsum += ls;
-                uint8_t *Pb = P + p * kPBuf;
-#pragma unroll
-                for (int g = 0; g < 4; ++g)
-                    *reinterpret_cast<uint4 *>(Pb + swz((uint32_t)hl, (uint32_t)(4 * u + g))) =
-                        make_uint4(pk[4 * g], pk[4 * g + 1], pk[4 * g + 2], pk[4 * g + 3]);
-                fence_async_smem();
-                tc_fence_before();
-            } else {
-                mbar_arrive(&ms.s_free[sb]);
-            }
-            mbar_arrive(&ms.p_full[p]);
-        }
+        for (int t = 0; t < nh; ++t) softmax_tile(t, false, m_run, lsum);
         // softmax denominators: the two halves of each head
         if (bar_and(1, kSoftmax, ok)) {
             lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);
