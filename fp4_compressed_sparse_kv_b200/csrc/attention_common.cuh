@@ -129,24 +129,25 @@ __device__ __forceinline__ void dequant16(const EntryRef &r, int lane, float *v)
     if (!r.swa) {
         const uint2 c = reinterpret_cast<const uint2 *>(r.p)[lane];
         const float s = e4m3_to_f32(r.sc[lane]);
-        const uint32_t cw[2] = {c.x, c.y};
+        uint32_t h2[8];
+        e2m1x8_to_f16x2x4(c.x, h2);
+        e2m1x8_to_f16x2x4(c.y, h2 + 4);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const uint32_t h2 = e2m1x2_to_f16x2((uint8_t)((cw[i / 4] >> (8 * (i % 4))) & 0xFF));
-            v[2 * i] = h_lo(h2) * s;
-            v[2 * i + 1] = h_hi(h2) * s;
+            v[2 * i] = h_lo(h2[i]) * s;
+            v[2 * i + 1] = h_hi(h2[i]) * s;
         }
     } else {
         const uint4 c = reinterpret_cast<const uint4 *>(r.p)[lane];
         const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const uint32_t lo = e4m3x2_to_f16x2((uint16_t)(cw[i] & 0xFFFF));
-            const uint32_t hi = e4m3x2_to_f16x2((uint16_t)(cw[i] >> 16));
-            v[4 * i] = h_lo(lo) * r.fscale;
-            v[4 * i + 1] = h_hi(lo) * r.fscale;
-            v[4 * i + 2] = h_lo(hi) * r.fscale;
-            v[4 * i + 3] = h_hi(hi) * r.fscale;
+            uint32_t hv[2];
+            e4m3x4_to_f16x2x2(cw[i], hv);
+            v[4 * i] = h_lo(hv[0]) * r.fscale;
+            v[4 * i + 1] = h_hi(hv[0]) * r.fscale;
+            v[4 * i + 2] = h_lo(hv[1]) * r.fscale;
+            v[4 * i + 3] = h_hi(hv[1]) * r.fscale;
         }
     }
 }

@@ -28,8 +28,8 @@
 //
 // Warp roles (768 threads).
 //   warps 0-15  producers: thread (e, cp) dequantises channels 64cp .. 64cp+63 of entry e (V chunk
-//               cp) from raw bytes it loaded two tiles earlier, once PV has released the buffer;
-//               they also load Q and write O^T at the end;
+//               cp) into registers one tile ahead and stores them once PV has released the
+//               buffer; they also load Q and write O^T at the end;
 //   warps 16-19 softmax, warp 16+q on TMEM quarter q (heads 16q .. 16q+15): lane l reads row
 //               16q + l%16 of S_(l/16), trades halves with lane l^16 and owns entries 32(l/16) ..
 //               32(l/16)+31 of that head, so a head's maximum and sum need one shuffle;
@@ -174,12 +174,11 @@ __device__ __forceinline__ void split_halves(int units, int s, int splits, int &
 // Entry table: for each row e of each tile, the FP4 cache row (page * 64 + offset) of the entry,
 // -(slot + 2) for a window entry, or -1 for a masked row (past the split or the sequence).
 
-// A producer thread's share of one tile: entry e, channels 128cp .. 128cp+127 (V chunks 2cp,
-// 2cp+1).  The raw bytes of an FP4 entry (64 B of codes, 8 scale bytes, contiguous) are loaded
-// into registers two tiles before they are dequantised; a window entry (128 E4M3 values) is
-// read when it is written, since the window is at most two tiles of a sequence.  (A mapping in
-// which one warp-wide load covers two whole entries loads fewer lines but writes the swizzled
-// V rows with 4-way bank conflicts, which costs more.)
+// A producer thread's share of one tile: entry e, channels 64cp .. 64cp+63 (V chunk cp).  The raw
+// bytes of an FP4 entry (32 B of codes, 4 scale bytes) are loaded into registers two tiles ahead
+// and dequantised one tile ahead, so that once PV releases the buffer only the stores remain; a
+// window entry (64 E4M3 values) is read when it is dequantised, since the window is at most two
+// tiles of a sequence.
 struct RawHalf {
     uint4 code[2];
     uint32_t sc;
@@ -196,30 +195,28 @@ struct RawHalf {
         }
     }
 
-    // Dequantise into V chunk cp, row e.
-    __device__ __forceinline__ void write(const AttnArgs &a, uint8_t *Vb, int e, int cp) const
+    // Dequantise into v: channels 64cp .. 64cp+63 as 32 fp16 pairs (zeros for a masked row).
+    __device__ __forceinline__ void dequant(const AttnArgs &a, int cp, uint32_t *v) const
     {
-        uint8_t *dst = Vb + cp * kVChunk;
         if (row == -1) {
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj)
-                *reinterpret_cast<uint4 *>(dst + swz((uint32_t)e, (uint32_t)jj)) = make_uint4(0u, 0u, 0u, 0u);
+            for (int i = 0; i < 32; ++i) v[i] = 0u;
         } else if (row >= 0) {
+            uint32_t sh[2];   // the four group scales as (s0, s1), (s2, s3)
+            e4m3x4_to_f16x2x2(sc, sh);
 #pragma unroll
             for (int gg = 0; gg < 4; ++gg) {
-                const uint32_t sh = e4m3x2_to_f16x2((uint16_t)((sc >> (8 * gg)) & 0xFF));
-                const uint32_t s2 = (sh & 0xFFFFu) | (sh << 16);
+                // group gg's scale in both halves
+                const uint32_t s2 = __byte_perm(sh[gg >> 1], 0u, (gg & 1) ? 0x3232u : 0x1010u);
                 const uint4 cw = code[gg >> 1];
-                const uint32_t w0 = (gg & 1) ? cw.z : cw.x, w1 = (gg & 1) ? cw.w : cw.y;
-                uint32_t v[8];
+                uint32_t c0[4], c1[4];
+                e2m1x8_to_f16x2x4((gg & 1) ? cw.z : cw.x, c0);
+                e2m1x8_to_f16x2x4((gg & 1) ? cw.w : cw.y, c1);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    v[q] = hmul2_u32(e2m1x2_to_f16x2((uint8_t)(w0 >> (8 * q))), s2);
-                    v[4 + q] = hmul2_u32(e2m1x2_to_f16x2((uint8_t)(w1 >> (8 * q))), s2);
+                    v[8 * gg + q] = hmul2_u32(c0[q], s2);
+                    v[8 * gg + 4 + q] = hmul2_u32(c1[q], s2);
                 }
-                *reinterpret_cast<uint4 *>(dst + swz((uint32_t)e, (uint32_t)(2 * gg))) = make_uint4(v[0], v[1], v[2], v[3]);
-                *reinterpret_cast<uint4 *>(dst + swz((uint32_t)e, (uint32_t)(2 * gg + 1))) =
-                    make_uint4(v[4], v[5], v[6], v[7]);
             }
         } else {
             // window entry: 64 E4M3 values times the entry's binary32 scale, rounded to fp16
@@ -230,20 +227,27 @@ struct RawHalf {
             for (int q = 0; q < 4; ++q) {
                 const uint4 w = src[q];
                 const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-                uint32_t v[8];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    const uint32_t lo = e4m3x2_to_f16x2((uint16_t)(ww[k] & 0xFFFF));
-                    const uint32_t hi = e4m3x2_to_f16x2((uint16_t)(ww[k] >> 16));
-                    v[2 * k] = pack_f16x2(h_lo(lo) * fs, h_hi(lo) * fs);
-                    v[2 * k + 1] = pack_f16x2(h_lo(hi) * fs, h_hi(hi) * fs);
+                    uint32_t hv[2];
+                    e4m3x4_to_f16x2x2(ww[k], hv);
+                    v[8 * q + 2 * k] = pack_f16x2(h_lo(hv[0]) * fs, h_hi(hv[0]) * fs);
+                    v[8 * q + 2 * k + 1] = pack_f16x2(h_lo(hv[1]) * fs, h_hi(hv[1]) * fs);
                 }
-                *reinterpret_cast<uint4 *>(dst + swz((uint32_t)e, (uint32_t)(2 * q))) = make_uint4(v[0], v[1], v[2], v[3]);
-                *reinterpret_cast<uint4 *>(dst + swz((uint32_t)e, (uint32_t)(2 * q + 1))) = make_uint4(v[4], v[5], v[6], v[7]);
             }
         }
     }
 };
+
+// Row e of V chunk cp: 8 swizzled 16-byte units.
+__device__ __forceinline__ void store_row(uint8_t *Vb, int e, int cp, const uint32_t *v)
+{
+    uint8_t *dst = Vb + cp * kVChunk;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        *reinterpret_cast<uint4 *>(dst + swz((uint32_t)e, (uint32_t)j)) =
+            make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+}
 
 // Fill the entry table with tiles t0 .. t0 + kTabHalves - 1: thread i (of the first kTabFill
 // producers) takes unit i of the range (8 entries: one selected block, or 8 window positions), so
@@ -562,7 +566,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_split_tc_kernel(AttnArgs a
         dummy.row = 0;
         dummy.code[0] = dummy.code[1] = make_uint4(0u, 0u, 0u, 0u);
         dummy.sc = 0x38383838u;   // E4M3 1.0
-        dummy.write(a, V + 2 * kVBuf, threadIdx.x & (kHalf - 1), threadIdx.x >> 6);
+        uint32_t v[32];
+        dummy.dequant(a, threadIdx.x >> 6, v);
+        store_row(V + 2 * kVBuf, threadIdx.x & (kHalf - 1), threadIdx.x >> 6, v);
     }
     grid_dep_wait();   // the selected blocks of the previous grid
 
@@ -656,16 +662,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_split_tc_kernel(AttnArgs a
         RawHalf raw0, raw1;   // tiles of even and of odd index
         raw0.fetch(a, tab[e], cp);
         if (nh > 1) raw1.fetch(a, tab[kHalf + e], cp);
-        auto step = [&](int t, RawHalf &rw) {
+        uint32_t v[32];       // the next tile's row, dequantised before its buffer is free
+        raw0.dequant(a, cp, v);
+        // rw holds tile t, already dequantised into v, so it takes tile t + 2 at once; rn holds t + 1
+        auto step = [&](int t, RawHalf &rw, const RawHalf &rn) {
             const int p = t % kStages;
-            if (t >= kStages) ok = ok && warp_wait(&ms.v_free[p], (uint32_t)(t / kStages - 1) & 1u, &ms.abort_flag, a.ws, 5);
-            if (ok) rw.write(a, V + p * kVBuf, e, cp);
-            if (cp == 0) {
-                const unsigned int vb = __ballot_sync(0xffffffffu, rw.row != -1);
-                if (lane == 0) reinterpret_cast<volatile uint32_t *>(&ms.vmask[p])[warp] = vb;
-            }
-            fence_async_smem();
-            warp_arrive(&ms.v_ready[p]);
+            const unsigned int vb = __ballot_sync(0xffffffffu, rw.row != -1);   // tile t's valid rows
             if (t + 2 < nh) {
                 if ((t + 2) % kTabHalves == 0) {
                     // the next tiles' entry addresses (every producer has fetched from the old ones)
@@ -675,11 +677,17 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_split_tc_kernel(AttnArgs a
                 }
                 rw.fetch(a, tab[((t + 2) % kTabHalves) * kHalf + e], cp);
             }
+            if (t >= kStages) ok = ok && warp_wait(&ms.v_free[p], (uint32_t)(t / kStages - 1) & 1u, &ms.abort_flag, a.ws, 5);
+            if (ok) store_row(V + p * kVBuf, e, cp, v);
+            if (cp == 0 && lane == 0) reinterpret_cast<volatile uint32_t *>(&ms.vmask[p])[warp] = vb;
+            fence_async_smem();
+            warp_arrive(&ms.v_ready[p]);
+            if (t + 1 < nh) rn.dequant(a, cp, v);
         };
 #pragma unroll 1
         for (int t = 0; t < nh; t += 2) {
-            step(t, raw0);
-            if (t + 1 < nh) step(t + 1, raw1);
+            step(t, raw0, raw1);
+            if (t + 1 < nh) step(t + 1, raw1, raw0);
         }
     } else {
         // ------------------------------- softmax -------------------------------

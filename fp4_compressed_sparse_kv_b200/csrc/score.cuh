@@ -72,9 +72,9 @@ __device__ __forceinline__ float score_key(const Q &q2, const float (&w)[8], uin
     const uint32_t kw[4] = {kr.x, kr.y, kr.z, kr.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const uint32_t lo = e4m3x2_to_f16x2((uint16_t)(kw[i] & 0xFFFF));
-        const uint32_t hi = e4m3x2_to_f16x2((uint16_t)(kw[i] >> 16));
-        const float k0 = h_lo(lo), k1 = h_hi(lo), k2v = h_lo(hi), k3 = h_hi(hi);
+        uint32_t hv[2];
+        e4m3x4_to_f16x2x2(kw[i], hv);
+        const float k0 = h_lo(hv[0]), k1 = h_hi(hv[0]), k2v = h_lo(hv[1]), k3 = h_hi(hv[1]);
         k2[4 * i + 0] = f2_pack(k0, k0);
         k2[4 * i + 1] = f2_pack(k1, k1);
         k2[4 * i + 2] = f2_pack(k2v, k2v);
