@@ -208,6 +208,7 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const float *__restri
     __shared__ float red[8];
     const int h = blockIdx.x, b = blockIdx.y, t = threadIdx.x, lane = t & 31, warp = t >> 5;
     grid_dep_wait();   // every split's partial
+    grid_dep_launch();   // a dependent kernel launched after this one waits for it before reading
     // the partials of the first kPre splits are loaded at once, before (and independently of) the
     // split weights, so that the whole read is one round trip
     constexpr int kPre = 24;

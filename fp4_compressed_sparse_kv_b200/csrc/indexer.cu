@@ -248,6 +248,10 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_kernel(const float *__re
     __shared__ uint32_t wcount[2][kTopkWarps];
     __shared__ uint32_t sel[2];
     const int b = blockIdx.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    // the next kernel (the attention) may start its own preparation while the selection runs; the
+    // scores are read only once the previous grid (the block scorer) has finished
+    grid_dep_launch();
+    grid_dep_wait();
     const int L = seq_len[b];
     int n;
     if (L < 1 || L > max_seq_len) {
@@ -320,6 +324,10 @@ __global__ void reuse_kernel(const int32_t *__restrict__ prev, const int32_t *__
                              int32_t *__restrict__ out, int32_t *__restrict__ out_count, int out_cap, void *ws)
 {
     const int b = blockIdx.x;
+    // the next kernel (the layer's attention) may start its own preparation while this copy runs;
+    // the previous layer's set is read only once the previous grid has finished
+    grid_dep_launch();
+    grid_dep_wait();
     int n = prev_count[b];
     if (n < 0 || n > prev_cap || n > out_cap) {
         if (threadIdx.x == 0) report(ws, CSA_ERR_DEVICE_DATA, b);
@@ -393,16 +401,15 @@ cudaError_t launch_topk(const float *scores, int score_stride, const int32_t *se
         (size_t)kTopkHistWords * 4 + (size_t)(max_candidates < kTopkCacheKeys ? max_candidates : kTopkCacheKeys) * 4;
     cudaError_t e = allow_dynamic_smem(reinterpret_cast<const void *>(topk_kernel), smem);
     if (e != cudaSuccess) return e;
-    topk_kernel<<<B, kTopkThreads, smem, st>>>(scores, score_stride, seq_len, max_seq_len, pool, pool_count, pool_cap,
-                                               k, out_blocks, out_count, ws);
-    return cudaGetLastError();
+    return launch_overlapped(topk_kernel, dim3(B), dim3(kTopkThreads), smem, st, scores, score_stride, seq_len,
+                             max_seq_len, pool, pool_count, pool_cap, k, out_blocks, out_count, ws);
 }
 
 cudaError_t launch_reuse(int B, const int32_t *prev, const int32_t *prev_count, int prev_cap, int32_t *out,
                          int32_t *out_count, int out_cap, void *ws, cudaStream_t st)
 {
-    reuse_kernel<<<B, 256, 0, st>>>(prev, prev_count, prev_cap, out, out_count, out_cap, ws);
-    return cudaGetLastError();
+    return launch_overlapped(reuse_kernel, dim3(B), dim3(256), 0, st, prev, prev_count, prev_cap, out, out_count,
+                             out_cap, ws);
 }
 
 }  // namespace csa

@@ -22,6 +22,7 @@
 
 #include "common.cuh"
 #include "convert.cuh"
+#include "pipeline.cuh"
 
 namespace csa {
 
@@ -147,6 +148,9 @@ __global__ void __launch_bounds__(256) kv_pack_kernel(csa_kv_layer layer, const 
                                                       const float *__restrict__ norm_w,
                                                       const float *__restrict__ rope_cs)
 {
+    // a dependent kernel launched after this one (the indexer's query terms, an attention) may be
+    // scheduled now: each waits for this grid before it reads anything this grid writes
+    grid_dep_launch();
     const int tok0 = (blockIdx.x * 8 + (threadIdx.x >> 5)) * kPackTok;
     const int lane = threadIdx.x & 31;
     PackIn in[kPackTok];
