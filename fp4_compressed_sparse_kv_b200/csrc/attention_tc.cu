@@ -45,9 +45,9 @@
 namespace csa {
 
 constexpr int kTcHeads = 64;
-constexpr int kHalf = 64;                        // entries per tile
-constexpr int kHalfUnits = kHalf / kAttnUnit;    // 8 units of 8 entries
-constexpr int kTcUnits = 2 * kHalfUnits;         // units per 128 entries (split sizing)
+constexpr int kTile = 64;                        // entries per tile
+constexpr int kTileUnits = kTile / kAttnUnit;    // 8 units of 8 entries
+constexpr int kTcUnits = 2 * kTileUnits;         // units per 128 entries (split sizing)
 constexpr int kTcChunks = kLatent / 64;          // 8 chunks of 64 channels
 constexpr int kStages = 3;                       // tiles in flight
 constexpr int kProducers = 512;                  // warps 0-15
@@ -55,14 +55,14 @@ constexpr int kSoftmax = 128;                    // warps 16-19
 constexpr int kSoftmaxWarp = 16;
 constexpr int kIssuerWarp = 20;                  // warps 20-23
 constexpr int kTcThreads = 768;
-constexpr uint32_t kVChunk = kHalf * 128;        // 8 KB: 64 rows x 64 fp16
+constexpr uint32_t kVChunk = kTile * 128;        // 8 KB: 64 rows x 64 fp16
 constexpr uint32_t kVBuf = kTcChunks * kVChunk;  // 64 KB per tile buffer
 constexpr uint32_t kPBuf = kTcHeads * 128;       // 8 KB: 64 head rows x 64 entries fp16
-constexpr int kTabHalves = 32;                   // tiles of entry addresses resolved at a time
+constexpr int kTabTiles = 32;                    // tiles of entry addresses resolved at a time
 constexpr uint32_t kOffV = 0;
 constexpr uint32_t kOffP = kOffV + kStages * kVBuf;
 constexpr uint32_t kOffTab = kOffP + kStages * kPBuf;
-constexpr uint32_t kOffMisc = kOffTab + kTabHalves * kHalf * 4;
+constexpr uint32_t kOffMisc = kOffTab + kTabTiles * kTile * 4;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0;                    // O^T: M-tile m in columns 64m .. 64m+63
 constexpr uint32_t kColQ = 256;                  // Q_x: 128 columns in lane half x
@@ -89,7 +89,7 @@ struct TcMisc {
 
 constexpr size_t kTcSmem = kOffMisc + sizeof(TcMisc) + 1024;
 
-constexpr uint32_t kIdescQK = umma_idesc_f16(64, kHalf, false, false);
+constexpr uint32_t kIdescQK = umma_idesc_f16(64, kTile, false, false);
 constexpr uint32_t kIdescPV = umma_idesc_f16(128, kTcHeads, true, false);
 
 __device__ __forceinline__ uint32_t swz(uint32_t row, uint32_t unit) { return row * 128u + ((unit ^ (row & 7u)) << 4); }
@@ -147,28 +147,14 @@ __device__ __forceinline__ void tc_ld16_sync(uint32_t taddr, float *v)
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-__device__ __forceinline__ void tc_st16(uint32_t taddr, const float *v)
-{
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
-        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
-        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
-        "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
-        "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
-        "r"(__float_as_uint(v[15]))
-        : "memory");
-}
-
 // Tile-aligned split of a sequence's units: split s of `splits` gets whole 8-unit tiles, so every
 // tile but the sequence's last is full.
-__device__ __forceinline__ void split_halves(int units, int s, int splits, int &ub, int &ue)
+__device__ __forceinline__ void split_tiles(int units, int s, int splits, int &ub, int &ue)
 {
-    const int halves = (units + kHalfUnits - 1) / kHalfUnits;
-    const int hb = (int)((long long)halves * s / splits), he = (int)((long long)halves * (s + 1) / splits);
-    ub = hb * kHalfUnits;
-    ue = he * kHalfUnits < units ? he * kHalfUnits : units;
+    const int tiles = (units + kTileUnits - 1) / kTileUnits;
+    const int hb = (int)((long long)tiles * s / splits), he = (int)((long long)tiles * (s + 1) / splits);
+    ub = hb * kTileUnits;
+    ue = he * kTileUnits < units ? he * kTileUnits : units;
 }
 
 // Entry table: for each row e of each tile, the FP4 cache row (page * 64 + offset) of the entry,
@@ -179,7 +165,7 @@ __device__ __forceinline__ void split_halves(int units, int s, int splits, int &
 // and dequantised one tile ahead, so that once PV releases the buffer only the stores remain; a
 // window entry (64 E4M3 values) is read when it is dequantised, since the window is at most two
 // tiles of a sequence.
-struct RawHalf {
+struct RawEntry {
     uint4 code[2];
     uint32_t sc;
     int32_t row;
@@ -249,15 +235,15 @@ __device__ __forceinline__ void store_row(uint8_t *Vb, int e, int cp, const uint
             make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
 }
 
-// Fill the entry table with tiles t0 .. t0 + kTabHalves - 1: thread i (of the first kTabFill
+// Fill the entry table with tiles t0 .. t0 + kTabTiles - 1: thread i (of the first kTabFill
 // producers) takes unit i of the range (8 entries: one selected block, or 8 window positions), so
 // the block id and the page table are read once per unit, in two rounds of independent loads.
-constexpr int kTabFill = kTabHalves * kHalfUnits;
+constexpr int kTabFill = kTabTiles * kTileUnits;
 static_assert(kTabFill <= kProducers, "one unit of the table per filling thread");
 __device__ __forceinline__ void fill_table(const AttnArgs &a, TcMisc &ms, int32_t *tab, int t0, int tid)
 {
     const SeqView &sv = ms.sv;
-    const int u = ms.u_begin + t0 * kHalfUnits + tid;
+    const int u = ms.u_begin + t0 * kTileUnits + tid;
     int32_t *out = tab + tid * kAttnUnit;
     int32_t code = -1;         // code of position 0 of the unit, or -1 for none
     int limit = 0;             // positions j < limit of the unit are valid
@@ -562,24 +548,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_split_tc_kernel(AttnArgs a
         float dm = kNoMax, dl = 0.f;
         softmax_tile(0, true, dm, dl);
     } else if (warp < kSoftmaxWarp) {
-        RawHalf dummy;
+        RawEntry dummy;
         dummy.row = 0;
         dummy.code[0] = dummy.code[1] = make_uint4(0u, 0u, 0u, 0u);
         dummy.sc = 0x38383838u;   // E4M3 1.0
         uint32_t v[32];
         dummy.dequant(a, threadIdx.x >> 6, v);
-        store_row(V + 2 * kVBuf, threadIdx.x & (kHalf - 1), threadIdx.x >> 6, v);
+        store_row(V + 2 * kVBuf, threadIdx.x & (kTile - 1), threadIdx.x >> 6, v);
     }
     grid_dep_wait();   // the selected blocks of the previous grid
 
     if (threadIdx.x == 0) {
         int ub = 0, ue = 0;
-        if (seq_view(a, b, ms.sv)) split_halves(ms.sv.units, s, a.splits, ub, ue);
+        if (seq_view(a, b, ms.sv)) split_tiles(ms.sv.units, s, a.splits, ub, ue);
         ms.u_begin = ub;
         ms.u_end = ue;
     }
     __syncthreads();
-    const int nh = (ms.u_end - ms.u_begin + kHalfUnits - 1) / kHalfUnits;   // tiles of this split
+    const int nh = (ms.u_end - ms.u_begin + kTileUnits - 1) / kTileUnits;   // tiles of this split
     if (threadIdx.x < kTabFill && nh > 0) fill_table(a, ms, tab, 0, threadIdx.x);
     __syncthreads();
 
@@ -638,7 +624,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_split_tc_kernel(AttnArgs a
 #pragma unroll
                     for (int mi = 0; mi < 2; ++mi)
 #pragma unroll
-                        for (int kk = 0; kk < kHalf / 16; ++kk) {
+                        for (int kk = 0; kk < kTile / 16; ++kk) {
                             const int m = m0 + mi;
                             const uint64_t ad = umma_sdesc_sw128(sV + p * kVBuf + 2 * m * kVChunk + kk * 2048, kVChunk, 1024);
                             const uint64_t bd = umma_sdesc_sw128(sP + p * kPBuf + kk * 32, 16, 1024);
@@ -658,24 +644,24 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_split_tc_kernel(AttnArgs a
         // ------------------------------- producers -------------------------------
         // After a failed wait the loop still runs to the end, skipping the work, so that every
         // producer takes the same barriers (the entry-table refills).
-        const int d = threadIdx.x, e = d & (kHalf - 1), cp = d >> 6;
-        RawHalf raw0, raw1;   // tiles of even and of odd index
+        const int d = threadIdx.x, e = d & (kTile - 1), cp = d >> 6;
+        RawEntry raw0, raw1;   // tiles of even and of odd index
         raw0.fetch(a, tab[e], cp);
-        if (nh > 1) raw1.fetch(a, tab[kHalf + e], cp);
+        if (nh > 1) raw1.fetch(a, tab[kTile + e], cp);
         uint32_t v[32];       // the next tile's row, dequantised before its buffer is free
         raw0.dequant(a, cp, v);
         // rw holds tile t, already dequantised into v, so it takes tile t + 2 at once; rn holds t + 1
-        auto step = [&](int t, RawHalf &rw, const RawHalf &rn) {
+        auto step = [&](int t, RawEntry &rw, const RawEntry &rn) {
             const int p = t % kStages;
             const unsigned int vb = __ballot_sync(0xffffffffu, rw.row != -1);   // tile t's valid rows
             if (t + 2 < nh) {
-                if ((t + 2) % kTabHalves == 0) {
+                if ((t + 2) % kTabTiles == 0) {
                     // the next tiles' entry addresses (every producer has fetched from the old ones)
                     bar_sync(3, kProducers);
                     if (d < kTabFill) fill_table(a, ms, tab, t + 2, d);
                     bar_sync(3, kProducers);
                 }
-                rw.fetch(a, tab[((t + 2) % kTabHalves) * kHalf + e], cp);
+                rw.fetch(a, tab[((t + 2) % kTabTiles) * kTile + e], cp);
             }
             if (t >= kStages) ok = ok && warp_wait(&ms.v_free[p], (uint32_t)(t / kStages - 1) & 1u, &ms.abort_flag, a.ws, 5);
             if (ok) store_row(V + p * kVBuf, e, cp, v);
