@@ -242,6 +242,10 @@ csa_status csa_index_reuse(int32_t B, const int32_t *prev_blocks, const int32_t 
  * (exact for these values) and fp32 accumulation; agrees with exact arithmetic to within
  * 2e-3 of max|out| per sequence.  With H = 64 or 128 the caches may hold at most 2^31 FP4 entries
  * (num_pages * 64) and 2^30 window entries (num_rows * 128); larger layers return CSA_ERR_UNSUPPORTED.
+ * Stream order: the call may begin while the stream's previous kernel is still running, when that
+ * kernel releases its dependents early (this library's kernels do), and it reads q at that point;
+ * everything else it reads only after the previous kernel has completed.  So q must not be written
+ * by an immediately preceding kernel that releases its dependents early (a plain launch does not).
  */
 csa_status csa_sparse_decode_attn(const csa_kv_layer *layer, const csa_batch *batch,
                                   const uint16_t *q, int32_t H, float sm_scale,
