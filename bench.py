@@ -141,8 +141,8 @@ KERNEL_SOURCES = {"indexer_full": ["screen.cu", "select.cu", "score.cuh", "radix
                                       "pipeline.cuh"],
                   "sparse_decode_attn": ["attention_cc.cu", "attention_tc.cu", "attention_common.cuh", "tcgen05.cuh",
                                          "common.cuh", "convert.cuh", "pipeline.cuh"],
-                  "kv_pack_fp4": ["pack.cu", "common.cuh", "convert.cuh"],
-                  "kv_pack_fp4_prefill": ["pack.cu", "common.cuh", "convert.cuh"]}
+                  "kv_pack_fp4": ["pack.cu", "common.cuh", "convert.cuh", "pipeline.cuh"],
+                  "kv_pack_fp4_prefill": ["pack.cu", "common.cuh", "convert.cuh", "pipeline.cuh"]}
 
 
 def traffic_from_profiles(call, workload):
