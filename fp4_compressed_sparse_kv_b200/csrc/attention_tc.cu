@@ -30,9 +30,10 @@
 //   warps 0-15  producers: thread (e, cp) dequantises channels 64cp .. 64cp+63 of entry e (V chunk
 //               cp) into registers one tile ahead and stores them once PV has released the
 //               buffer; they also load Q and write O^T at the end;
-//   warps 16-19 softmax, warp 16+q on TMEM quarter q (heads 16q .. 16q+15): lane l reads row
-//               16q + l%16 of S_(l/16), trades halves with lane l^16 and owns entries 32(l/16) ..
-//               32(l/16)+31 of that head, so a head's maximum and sum need one shuffle;
+//   warps 16-19 softmax, warp 16+q on TMEM quarter q (heads 16q .. 16q+15): lane l owns entries
+//               32(l/16) .. 32(l/16)+31 of head 16q + l%16 and reads both channel halves' scores of
+//               them with 16-lane loads split between the half-warps, so a head's maximum and sum
+//               need one shuffle (with lane l^16, which owns the head's other 32 entries);
 //   warps 20-23 MMA issuers (lane 0): 20, 21 = QK of channel half 0, 1 (warp 20 also owns the TMEM
 //               allocation); 22, 23 = PV of M-tiles 0-1, 2-3.  Two issuers per product, because one
 //               thread issues a tcgen05.mma only every ~65 cycles, twice what an M=64 MMA takes.
